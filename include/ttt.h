@@ -1,0 +1,172 @@
+/*
+ * ttt.h -- C ABI of the B200 large-chunk test-time-training (TTT) layer.
+ *
+ * The layer keeps, per head, SwiGLU fast weights
+ *     f_W(x) = W2 (SiLU(W1 x) o (W3 x)),   W1, W3 in R^{m x d},  W2 in R^{d x m}
+ * (ZipMap: Linear-Time Stateful 3D Reconstruction via Test-Time Training,
+ * key design 1), takes one or more Muon steps of the per-token-weighted
+ * dot-product loss
+ *     L = sum_i eta_i * ( - f_W(k_i)^T v_i )
+ * over every token of a chunk (Scal3R: Scalable Test-Time Training for
+ * Large-Scale 3D Reconstruction, scheme 1, eq. (9)), with the gradient
+ * orthogonalised by Newton-Schulz and a norm-preserving step
+ *     Delta <- NewtonSchulz(g),  W^ <- ||W|| (W - lr Delta) / ||W - lr Delta||
+ * (ZipMap key design 3), and then applies o_i = f_W^(q_i) (Scal3R eq. (4)).
+ * Options: L2-normalised Q/K and a depthwise ShortConv2D on V (VGG-T3:
+ * Offline Feed-Forward 3D Reconstruction at Scale, key designs 1 and 2), two
+ * inner steps (VGG-T3 key design 3), causal chunk-to-chunk carry of W (ZipMap
+ * key design 4; LoGeR: Long-Context Geometric Reconstruction with Hybrid
+ * Memory, method overview).
+ *
+ * Conventions for every entry point:
+ *  - All pointers are DEVICE pointers unless stated otherwise; the caller
+ *    owns every buffer, including the workspace, and the library never
+ *    allocates device memory.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream).  Argument, alignment and workspace
+ *    errors are detected on the host and returned before anything is queued.
+ *    A failed kernel launch returns TTT_ERR_CUDA.  A device-side wait that
+ *    exceeds its time limit does not hang: the kernel records
+ *    TTT_ERR_TIMEOUT in the workspace status word (read it with
+ *    ttt_poll_status) and returns.
+ *  - Token matrices Q, K, V, O are row-major [T][ld] with head h in columns
+ *    [h*d, (h+1)*d); ld is the row stride in elements (0 means H*d, else
+ *    ld >= H*d).  In TTT_BF16 mode they are bfloat16 and must be 16-byte
+ *    aligned with ld a multiple of 8; in TTT_FP32 mode they are float.
+ *  - eta is float [T][H] (per-token, per-head learning rate), contiguous.
+ *  - Fast weights are float: W1, W3 [H][m][d], W2 [H][d][m], contiguous.
+ *    In TTT_BF16 mode the GEMMs read a bfloat16 copy of W that the library
+ *    writes into the workspace at the start of each call; W itself stays fp32.
+ *  - TTT_BF16 mode runs the tensor-core path and needs d in {128, 192} and
+ *    m a multiple of 64; TTT_FP32 mode runs fp32 CUDA-core kernels for any
+ *    d <= 256 and m a multiple of 32.  Other shapes return TTT_ERR_UNSUPPORTED.
+ *  - No entry point falls back to the CPU.
+ */
+#ifndef TTT_H
+#define TTT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_INVALID = -1,      /* bad argument: null pointer, non-positive size, ld < H*d, ... */
+  TTT_ERR_UNSUPPORTED = -2,  /* valid but not implemented: shape or dtype outside the table above */
+  TTT_ERR_WORKSPACE = -3,    /* workspace missing or smaller than ttt_workspace_bytes() */
+  TTT_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
+  TTT_ERR_TIMEOUT = -5,      /* a device-side wait gave up (reported through ttt_poll_status) */
+  TTT_ERR_ALIGN = -6         /* pointer or row stride violates the 16-byte alignment rule */
+} ttt_status;
+
+typedef enum { TTT_FP32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+/* Per-head fast-weight dimensions: H heads, head dim d, SwiGLU hidden width m. */
+typedef struct { int heads, d, m; } ttt_dims;
+
+/* fp32 device pointers: W1, W3 [H][m][d]; W2 [H][d][m]. */
+typedef struct { float *W1, *W3, *W2; } ttt_weights;
+
+/* Muon step (ZipMap key design 3).  For each per-head matrix G (g1, g3, g2):
+ *   X = G / (||G||_F + eps), on the wide orientation (rows <= cols);
+ *   iters times: A = X X^T, X <- a X + (b A + c A A) X;  Delta = X (original orientation).
+ *   iters = 0: Delta = G (plain gradient step).
+ *   renorm = 1: W <- ||W||_F (W - lr Delta) / ||W - lr Delta||_F;  renorm = 0: W <- W - lr Delta. */
+typedef struct { int iters; float a, b, c, eps, lr; int renorm; } ttt_ns_cfg;
+
+/* Row strides and the Q/K L2-normalisation switch (VGG-T3 key design 1):
+ * qk_l2norm = 1 makes update/grad use k^ = k / max(||k||, 1e-12) and apply use
+ * q^ likewise, per token and head, without modifying Q or K. */
+typedef struct { int qk_l2norm; int64_t ld_q, ld_k, ld_v, ld_o; } ttt_io_cfg;
+
+/* Workspace size in bytes for any call of this library with these dims, with
+ * at most T tokens per call (for ttt_chunked: at most `chunk` tokens per chunk).
+ * The workspace must be 256-byte aligned.  Returns 0 for invalid dims. */
+size_t ttt_workspace_bytes(ttt_dims dims, int64_t T, ttt_dtype dtype);
+
+/* Clear the status word of a workspace (asynchronously on `stream`). */
+int ttt_reset_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream` and return the workspace status word: TTT_OK or the
+ * first device-side error recorded since the last reset (TTT_ERR_TIMEOUT). */
+int ttt_poll_status(const void* ws, void* stream);
+
+/* In-place L2 normalisation of X [T][ld]: every (token, head) row of d values
+ * becomes x / max(||x||_2, 1e-12) (VGG-T3 key design 1). */
+int ttt_l2norm(void* X, int64_t T, ttt_dims dims, int64_t ld, ttt_dtype dtype, void* stream);
+
+/* ShortConv2D (VGG-T3 key design 2): V [N*h*w][ld_v] is viewed as the patch
+ * grid (N, h, w, C) with token t = (n*h + y)*w + x; each channel c is
+ * cross-correlated with taps[c] (float [C][3][3], device) with zero padding
+ * inside each frame, no bias; act = 1 applies SiLU.  Writes Vout [N*h*w][ld_out]
+ * (C columns; may not alias V).  C must be a multiple of 8. */
+int ttt_shortconv2d(const void* V, int64_t ld_v, void* Vout, int64_t ld_out, const float* taps,
+                    int N, int h, int w, int C, int act, ttt_dtype dtype, void* stream);
+
+/* Gradient of L w.r.t. (W1, W3, W2) summed over all T tokens, fp32, written to
+ * G = [g1 (H*m*d) | g3 (H*m*d) | g2 (H*d*m)] (same layouts as W).  Uses K and V as
+ * given (apply ttt_shortconv2d to V first if wanted); deterministic.
+ * This and ttt_step split ttt_update so that a caller can sum G across devices
+ * (Scal3R scheme 2, Global Context Synchronization) between the two. */
+int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T,
+             ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, float* G,
+             void* ws, size_t ws_bytes, void* stream);
+
+/* Muon step from a given gradient G (layout as in ttt_grad); updates W in place. */
+int ttt_step(ttt_weights W, const float* G, const ttt_ns_cfg* ns, ttt_dims dims, ttt_dtype dtype,
+             void* ws, size_t ws_bytes, void* stream);
+
+/* TTTUpdate: `steps` times { G = gradient over all T tokens at the current W; Muon step }.
+ * steps = 2 is VGG-T3's test-time scaling.  T = 0 leaves W unchanged. */
+int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, int steps,
+               const ttt_ns_cfg* ns, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype,
+               void* ws, size_t ws_bytes, void* stream);
+
+/* Apply: O[i] = f_W(q_i) for T query rows (Q and O may not alias). */
+int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
+              const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* Causal chunk carry over T tokens in chunks of `chunk` (the last may be shorter).
+ * order 0: O_c = f_{W_(c-1)}(Q_c), then W_c = TTTUpdate(W_(c-1); chunk c);
+ * order 1: update first, then apply with W_c.  W is carried in place, so calling
+ * again with the returned W resumes the stream. */
+int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, const float* eta, void* O,
+                int64_t T, int64_t chunk, int order, int steps, const ttt_ns_cfg* ns, ttt_dims dims,
+                const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* ttt_status_string(int status);
+
+/* Number of kernel launches the library queued since load (for launch accounting). */
+uint64_t ttt_launch_count(void);
+
+/* Per-kernel device timing.  While profiling is on, the library records a pair
+ * of CUDA events on the launch stream around each of its kernels (or kernel
+ * groups) and files the pair under one of the kinds below.  ttt_profile_query
+ * waits for the recorded events, adds their durations to the kind's totals and
+ * returns them; ttt_profile_reset clears the totals.  Host-thread safe; the
+ * events cost a few microseconds per launch, so leave profiling off when not
+ * measuring. */
+typedef enum {
+  TTT_PROF_GRAD = 0,    /* gradient kernel (tensor-core in bf16 mode) */
+  TTT_PROF_APPLY = 1,   /* apply kernel */
+  TTT_PROF_NS = 2,      /* Newton-Schulz iterations and the weight step */
+  TTT_PROF_NORM = 3,    /* Q/K row norms and ttt_l2norm */
+  TTT_PROF_CONV = 4,    /* ShortConv2D */
+  TTT_PROF_REDUCE = 5,  /* split-K reduction of the gradient partials */
+  TTT_PROF_SHADOW = 6,  /* bf16 copies of the fast weights */
+  TTT_PROF_KINDS = 7
+} ttt_prof_kind;
+
+int ttt_profile_enable(int on);
+int ttt_profile_reset(void);
+int ttt_profile_query(int kind, double* total_ms, uint64_t* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H */

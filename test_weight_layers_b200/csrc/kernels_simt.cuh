@@ -1,0 +1,529 @@
+// CUDA-core kernels: memory-bound preprocessing (row norms, L2 norm, ShortConv2D),
+// weight shadows, the deterministic split-K reduction, Newton-Schulz and the
+// Muon weight step, and the fp32-mode gradient/apply used when the layer runs
+// in full fp32 precision.
+#pragma once
+
+#include "common.cuh"
+
+namespace ttt {
+
+template <typename T>
+struct Vec16;  // 16-byte vector of T
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+};
+
+__device__ __forceinline__ void load16(const float* p, float (&v)[4]) {
+  float4 x = *reinterpret_cast<const float4*>(p);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[8]) {
+  uint4 x = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store16(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store16(__nv_bfloat16* p, const float (&v)[8]) {
+  uint4 x;
+  x.x = pack_bf16x2(v[0], v[1]);
+  x.y = pack_bf16x2(v[2], v[3]);
+  x.z = pack_bf16x2(v[4], v[5]);
+  x.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = x;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// L2 norms of (token, head) rows (VGG-T3 key design 1): one warp per token.
+// mode 0: write r[t*H + h] = 1 / max(||x||, 1e-12);  mode 1: scale X in place.
+
+template <typename T>
+__global__ void k_rownorm(T* X, int64_t ld, int64_t rows, int H, int d, float* r_out, int mode) {
+  constexpr int VN = Vec16<T>::N;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int nv = d / VN;
+  for (int64_t t = warp_id; t < rows; t += nwarps) {
+    T* row = X + t * ld;
+    for (int h = 0; h < H; ++h) {
+      float ss = 0.f;
+      for (int v = lane; v < nv; v += 32) {
+        float x[VN];
+        load16(row + h * d + v * VN, x);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) ss = fmaf(x[i], x[i], ss);
+      }
+      ss = warp_sum(ss);
+      const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+      if (mode == 0) {
+        if (lane == 0) r_out[t * H + h] = inv;
+      } else {
+        for (int v = lane; v < nv; v += 32) {
+          float x[VN];
+          load16(row + h * d + v * VN, x);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) x[i] *= inv;
+          store16(row + h * d + v * VN, x);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// ShortConv2D (VGG-T3 key design 2): depthwise 3x3 zero-padded cross-correlation
+// per frame on the (N, h, w, C) patch grid.  threadIdx.x picks a 16-byte channel
+// vector (its 9*VN taps stay in registers), the y-dimension walks tokens.
+
+template <typename T>
+__global__ void k_shortconv(const T* __restrict__ V, int64_t ldv, T* __restrict__ out, int64_t ldo,
+                            const float* __restrict__ taps, int N, int gh, int gw, int C, int act) {
+  constexpr int VN = Vec16<T>::N;
+  const int cv = blockIdx.x * blockDim.x + threadIdx.x;  // channel vector
+  if (cv * VN >= C) return;
+  const int c0 = cv * VN;
+  float w[9][VN];
+#pragma unroll
+  for (int i = 0; i < VN; ++i)
+#pragma unroll
+    for (int k = 0; k < 9; ++k) w[k][i] = taps[(c0 + i) * 9 + k];
+  const int64_t ntok = (int64_t)N * gh * gw;
+  for (int64_t t = (int64_t)blockIdx.y * blockDim.y + threadIdx.y; t < ntok; t += (int64_t)gridDim.y * blockDim.y) {
+    const int x = (int)(t % gw);
+    const int y = (int)((t / gw) % gh);
+    float acc[VN];
+#pragma unroll
+    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int dy = -1; dy <= 1; ++dy) {
+      if (y + dy < 0 || y + dy >= gh) continue;
+#pragma unroll
+      for (int dx = -1; dx <= 1; ++dx) {
+        if (x + dx < 0 || x + dx >= gw) continue;
+        float v[VN];
+        load16(V + (t + (int64_t)dy * gw + dx) * ldv + c0, v);
+        const int k = (dy + 1) * 3 + (dx + 1);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[k][i], v[i], acc[i]);
+      }
+    }
+    if (act == 1) {
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[i] = acc[i] / (1.0f + expf(-acc[i]));
+    }
+    store16(out + t * ldo + c0, acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bf16 shadows of the fp32 fast weights, laid out for the tensor-core kernels:
+//   Wsh rows [0, Hm): W1 [H][m][d];  [Hm, 2Hm): W3;  [2Hm, 3Hm): W2^T [H][m][d]
+//   W2b [H][d][m]  (W2 itself)
+
+__global__ void k_shadow(const float* __restrict__ W1, const float* __restrict__ W3, const float* __restrict__ W2,
+                         __nv_bfloat16* __restrict__ Wsh, __nv_bfloat16* __restrict__ W2b, int H, int d, int m) {
+  const int64_t n = (int64_t)H * m * d;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    Wsh[i] = __float2bfloat16_rn(W1[i]);
+    Wsh[n + i] = __float2bfloat16_rn(W3[i]);
+    // i indexes W2^T [h][j][k]  <-  W2 [h][k][j]
+    const int64_t h = i / ((int64_t)m * d);
+    const int64_t rem = i % ((int64_t)m * d);
+    const int64_t j = rem / d, k = rem % d;
+    Wsh[2 * n + i] = __float2bfloat16_rn(W2[(h * d + k) * m + j]);
+    W2b[i] = __float2bfloat16_rn(W2[i]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Deterministic split-K reduction: G[i] = sum_{s=0..S-1} P[s][i] in that order.
+
+__global__ void k_reduce_splits(const float* __restrict__ P, int S, int64_t n, float* __restrict__ G) {
+  const int64_t n4 = n / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(P)[i];
+    for (int s = 1; s < S; ++s) {
+      float4 v = reinterpret_cast<const float4*>(P + (int64_t)s * n)[i];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    reinterpret_cast<float4*>(G)[i] = acc;
+  }
+}
+
+// Fixed-shape block reduction (256 threads) -> deterministic.
+__device__ __forceinline__ float block_sum_256(float v, float* red) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 8; ++i) s += red[i];
+    red[8] = s;
+  }
+  __syncthreads();
+  return red[8];
+}
+
+// ---------------------------------------------------------------------------
+// Newton-Schulz (ZipMap key design 3) on the 3H per-head gradient matrices.
+// Matrix b < 2H is g1/g3 of shape (m, d); b >= 2H is g2 of shape (d, m).
+// X_b = orient(G_b) / (||G_b||_F + eps) has the wide shape (r, c), r = min(m, d).
+
+__device__ __forceinline__ void mat_shape(int b, int H, int d, int m, int& R, int& C) {
+  if (b < 2 * H) { R = m; C = d; } else { R = d; C = m; }
+}
+
+__global__ void __launch_bounds__(256) k_frob_norms(const float* __restrict__ src, int64_t n_per, float* __restrict__ out) {
+  __shared__ float red[9];
+  const float* p = src + (int64_t)blockIdx.x * n_per;
+  float s = 0.f;
+  for (int64_t i = threadIdx.x; i < n_per; i += 256) s = fmaf(p[i], p[i], s);
+  s = block_sum_256(s, red);
+  if (threadIdx.x == 0) out[blockIdx.x] = sqrtf(s);
+}
+
+__global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, const float* __restrict__ norms, int H,
+                          int d, int m, float eps) {
+  const int b = blockIdx.y;
+  int R, C;
+  mat_shape(b, H, d, m, R, C);
+  const bool tall = R > C;
+  const int64_t n = (int64_t)m * d;
+  const float sc = 1.0f / (norms[b] + eps);
+  const float* g = G + (int64_t)b * n;
+  float* x = X + (int64_t)b * n;
+  const int c = tall ? R : C;  // columns of X
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    // i indexes X (r, c) row-major
+    const int64_t xi = i / c, xj = i % c;
+    x[i] = (tall ? g[xj * C + xi] : g[i]) * sc;
+  }
+}
+
+// Batched C = alpha * A * op(B) + beta * Cin, fp32, 64x64 tiles, 256 threads.
+// A: [M][K] (lda), op(B) = B [K][N] (ldb) or, with TRANS_B, B^T with B [N][K].
+template <bool TRANS_B>
+__global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const float* __restrict__ A, int lda, int64_t sA,
+                                                  const float* __restrict__ B, int ldb, int64_t sB, float* __restrict__ C,
+                                                  int ldc, int64_t sC, const float* __restrict__ Cin, float alpha,
+                                                  float beta) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int b = blockIdx.z;
+  A += b * sA;
+  B += b * sB;
+  C += b * sC;
+  if (Cin) Cin += b * sC;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      const int kk = i & 15, mm = i >> 4;
+      const int gm = m0 + mm, gk = k0 + kk;
+      As[kk][mm] = (gm < M && gk < K) ? A[(int64_t)gm * lda + gk] : 0.f;
+      if (TRANS_B) {
+        const int gn = n0 + mm;
+        Bs[kk][mm] = (gn < N && gk < K) ? B[(int64_t)gn * ldb + gk] : 0.f;
+      }
+    }
+    if (!TRANS_B) {
+      for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+        const int nn = i & 63, kk = i >> 6;
+        const int gn = n0 + nn, gk = k0 + kk;
+        Bs[kk][nn] = (gn < N && gk < K) ? B[(int64_t)gk * ldb + gn] : 0.f;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gm = m0 + ty + 16 * i, gn = n0 + tx + 16 * j;
+      if (gm < M && gn < N) {
+        float v = alpha * acc[i][j];
+        if (Cin) v = fmaf(beta, Cin[(int64_t)gm * ldc + gn], v);
+        C[(int64_t)gm * ldc + gn] = v;
+      }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Muon weight step (ZipMap key design 3): W <- ||W|| (W - lr D) / ||W - lr D||.
+// D_b is read from X_b (wide orientation, transposed back for tall matrices),
+// or from G_b directly when Newton-Schulz is disabled (iters = 0).
+
+__device__ __forceinline__ float delta_at(const float* __restrict__ D, int b, int64_t i, int H, int d, int m,
+                                          bool from_x) {
+  const int64_t n = (int64_t)m * d;
+  if (!from_x) return D[(int64_t)b * n + i];
+  int R, C;
+  mat_shape(b, H, d, m, R, C);
+  if (R <= C) return D[(int64_t)b * n + i];
+  const int64_t ri = i / C, cj = i % C;  // W index (ri, cj) -> X (cj, ri), X has R columns
+  return D[(int64_t)b * n + cj * R + ri];
+}
+
+__device__ __forceinline__ float* mat_ptr(float* W1, float* W3, float* W2, int b, int H, int64_t n) {
+  return b < H ? W1 + (int64_t)b * n : (b < 2 * H ? W3 + (int64_t)(b - H) * n : W2 + (int64_t)(b - 2 * H) * n);
+}
+
+__global__ void __launch_bounds__(256) k_step_norms(float* W1, float* W3, float* W2, const float* __restrict__ D, int H,
+                                                    int d, int m, float lr, int from_x, float* __restrict__ out) {
+  __shared__ float red[9];
+  const int b = blockIdx.x;
+  const int64_t n = (int64_t)m * d;
+  const float* w = mat_ptr(W1, W3, W2, b, H, n);
+  float s0 = 0.f, s1 = 0.f;
+  for (int64_t i = threadIdx.x; i < n; i += 256) {
+    const float wi = w[i];
+    const float u = wi - lr * delta_at(D, b, i, H, d, m, from_x != 0);
+    s0 = fmaf(wi, wi, s0);
+    s1 = fmaf(u, u, s1);
+  }
+  s0 = block_sum_256(s0, red);
+  s1 = block_sum_256(s1, red);
+  if (threadIdx.x == 0) {
+    out[2 * b] = sqrtf(s0);
+    out[2 * b + 1] = sqrtf(s1);
+  }
+}
+
+__global__ void k_step_apply(float* W1, float* W3, float* W2, const float* __restrict__ D, int H, int d, int m, float lr,
+                             int from_x, int renorm, const float* __restrict__ norms) {
+  const int b = blockIdx.y;
+  const int64_t n = (int64_t)m * d;
+  float* w = mat_ptr(W1, W3, W2, b, H, n);
+  float sc = 1.f;
+  if (renorm) {
+    const float nu = norms[2 * b + 1];
+    sc = nu > 0.f ? norms[2 * b] / nu : 1.f;
+  }
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    w[i] = sc * (w[i] - lr * delta_at(D, b, i, H, d, m, from_x != 0));
+}
+
+// ---------------------------------------------------------------------------
+// fp32 mode: gradient of the dot-product loss on CUDA cores (exact fp32 math).
+// grid (m/32 slices, H, S); each CTA owns 32 rows of m and accumulates
+// g1, g3 (rows) and g2 (columns) for its token range in registers.
+
+constexpr int F32_MS = 32, F32_TT = 32;
+
+__global__ void __launch_bounds__(256) k_grad_f32(const float* __restrict__ K, int64_t ldk, const float* __restrict__ V,
+                                                  int64_t ldv, const float* __restrict__ eta, const float* __restrict__ rk,
+                                                  const float* __restrict__ W1, const float* __restrict__ W3,
+                                                  const float* __restrict__ W2, float* __restrict__ partial, int64_t T,
+                                                  int H, int d, int m, int S) {
+  constexpr int MS = F32_MS, TT = F32_TT, NQ = MS * 256 / 256;  // d <= 256 -> MS*d/256 <= 32
+  extern __shared__ float sm[];
+  const int slice = blockIdx.x, h = blockIdx.y, split = blockIdx.z, tid = threadIdx.x;
+  const int j0 = slice * MS;
+  float* w1 = sm;
+  float* w3 = w1 + MS * d;
+  float* w2 = w3 + MS * d;  // [d][MS]
+  float* kt = w2 + d * MS;  // [TT][d]
+  float* vt = kt + TT * d;
+  float* f1 = vt + TT * d;  // [TT][MS]
+  float* f3 = f1 + TT * MS;
+  float* fz = f3 + TT * MS;
+  float* ee = fz + TT * MS;  // [TT]
+  float* rr = ee + TT;       // [TT]
+  for (int i = tid; i < MS * d; i += 256) {
+    const int jj = i / d, kk = i % d;
+    w1[i] = W1[((int64_t)h * m + j0 + jj) * d + kk];
+    w3[i] = W3[((int64_t)h * m + j0 + jj) * d + kk];
+  }
+  for (int i = tid; i < d * MS; i += 256) {
+    const int kk = i / MS, jj = i % MS;
+    w2[i] = W2[((int64_t)h * d + kk) * m + j0 + jj];
+  }
+  float a1[NQ], a3[NQ], a2[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) a1[q] = a3[q] = a2[q] = 0.f;
+  const int64_t tiles = (T + TT - 1) / TT;
+  const int64_t tb = tiles * split / S, te = tiles * (split + 1) / S;
+  const int nacc = MS * d;
+  for (int64_t tile = tb; tile < te; ++tile) {
+    const int64_t t0 = tile * TT;
+    __syncthreads();
+    for (int i = tid; i < TT * d; i += 256) {
+      const int t = i / d, kk = i % d;
+      const bool in = t0 + t < T;
+      kt[i] = in ? K[(t0 + t) * ldk + (int64_t)h * d + kk] : 0.f;
+      vt[i] = in ? V[(t0 + t) * ldv + (int64_t)h * d + kk] : 0.f;
+    }
+    if (tid < TT) {
+      const bool in = t0 + tid < T;
+      ee[tid] = in ? eta[(t0 + tid) * H + h] : 0.f;
+      rr[tid] = in ? (rk ? rk[(t0 + tid) * H + h] : 1.f) : 0.f;
+    }
+    __syncthreads();
+    for (int o = tid; o < 3 * TT * MS; o += 256) {
+      const int mat = o / (TT * MS), rem = o % (TT * MS), t = rem / MS, j = rem % MS;
+      float acc = 0.f;
+      if (mat == 0) {
+        for (int kk = 0; kk < d; ++kk) acc = fmaf(kt[t * d + kk], w1[j * d + kk], acc);
+        f1[rem] = acc;
+      } else if (mat == 1) {
+        for (int kk = 0; kk < d; ++kk) acc = fmaf(kt[t * d + kk], w3[j * d + kk], acc);
+        f3[rem] = acc;
+      } else {
+        for (int kk = 0; kk < d; ++kk) acc = fmaf(vt[t * d + kk], w2[kk * MS + j], acc);
+        fz[rem] = acc;
+      }
+    }
+    __syncthreads();
+    for (int o = tid; o < TT * MS; o += 256) {
+      const int t = o / MS;
+      const float r = rr[t], e = ee[t];
+      const float h1 = f1[o] * r, h3 = f3[o] * r, z = fz[o];
+      const float s = 1.0f / (1.0f + expf(-h1));
+      const float a = h1 * s, u = a * h3, du = -e * z;
+      f1[o] = du * h3 * s * (1.0f + h1 * (1.0f - s)) * r;  // dL/dh1, chained to the raw key
+      f3[o] = du * a * r;                                   // dL/dh3
+      fz[o] = -e * u;                                       // -eta u, the g2 factor
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = tid + 256 * q;
+      if (e < nacc) {
+        const int jj = e / d, kk = e % d;
+        float s1 = a1[q], s3 = a3[q];
+        for (int t = 0; t < TT; ++t) {
+          const float kv = kt[t * d + kk];
+          s1 = fmaf(f1[t * MS + jj], kv, s1);
+          s3 = fmaf(f3[t * MS + jj], kv, s3);
+        }
+        a1[q] = s1;
+        a3[q] = s3;
+        const int kk2 = e / MS, jj2 = e % MS;
+        float s2 = a2[q];
+        for (int t = 0; t < TT; ++t) s2 = fmaf(vt[t * d + kk2], fz[t * MS + jj2], s2);
+        a2[q] = s2;
+      }
+    }
+  }
+  const int64_t n = (int64_t)m * d;
+  float* p1 = partial + ((int64_t)split * 3 + 0) * H * n + (int64_t)h * n;
+  float* p3 = partial + ((int64_t)split * 3 + 1) * H * n + (int64_t)h * n;
+  float* p2 = partial + ((int64_t)split * 3 + 2) * H * n + (int64_t)h * n;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int e = tid + 256 * q;
+    if (e < nacc) {
+      const int jj = e / d, kk = e % d;
+      p1[(int64_t)(j0 + jj) * d + kk] = a1[q];
+      p3[(int64_t)(j0 + jj) * d + kk] = a3[q];
+      const int kk2 = e / MS, jj2 = e % MS;
+      p2[(int64_t)kk2 * m + j0 + jj2] = a2[q];
+    }
+  }
+}
+
+// fp32 mode apply: grid (ceil(T/32), H); O[t] = W2 (SiLU(W1 q^) o (W3 q^)).
+__global__ void __launch_bounds__(256) k_apply_f32(const float* __restrict__ Q, int64_t ldq, const float* __restrict__ rq,
+                                                   const float* __restrict__ W1, const float* __restrict__ W3,
+                                                   const float* __restrict__ W2, float* __restrict__ O, int64_t ldo,
+                                                   int64_t T, int H, int d, int m) {
+  constexpr int TT = F32_TT, MC = F32_MS, NQ = 32;  // TT*d/256 <= 32
+  extern __shared__ float sm[];
+  const int h = blockIdx.y, tid = threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.x * TT;
+  float* qt = sm;             // [TT][d]
+  float* w1 = qt + TT * d;    // [MC][d]
+  float* w3 = w1 + MC * d;    // [MC][d]
+  float* w2 = w3 + MC * d;    // [d][MC]
+  float* p = w2 + d * MC;     // [TT][MC]
+  float* rr = p + TT * MC;    // [TT]
+  for (int i = tid; i < TT * d; i += 256) {
+    const int t = i / d, kk = i % d;
+    qt[i] = (t0 + t < T) ? Q[(t0 + t) * ldq + (int64_t)h * d + kk] : 0.f;
+  }
+  if (tid < TT) rr[tid] = (t0 + tid < T) ? (rq ? rq[(t0 + tid) * H + h] : 1.f) : 0.f;
+  float acc[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+  const int nacc = TT * d;
+  for (int mc = 0; mc < m; mc += MC) {
+    __syncthreads();
+    for (int i = tid; i < MC * d; i += 256) {
+      const int jj = i / d, kk = i % d;
+      w1[i] = W1[((int64_t)h * m + mc + jj) * d + kk];
+      w3[i] = W3[((int64_t)h * m + mc + jj) * d + kk];
+    }
+    for (int i = tid; i < d * MC; i += 256) {
+      const int kk = i / MC, jj = i % MC;
+      w2[i] = W2[((int64_t)h * d + kk) * m + mc + jj];
+    }
+    __syncthreads();
+    for (int o = tid; o < TT * MC; o += 256) {
+      const int t = o / MC, j = o % MC;
+      float h1 = 0.f, h3 = 0.f;
+      for (int kk = 0; kk < d; ++kk) {
+        h1 = fmaf(qt[t * d + kk], w1[j * d + kk], h1);
+        h3 = fmaf(qt[t * d + kk], w3[j * d + kk], h3);
+      }
+      h1 *= rr[t];
+      h3 *= rr[t];
+      p[o] = h1 / (1.0f + expf(-h1)) * h3;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = tid + 256 * q;
+      if (e < nacc) {
+        const int t = e / d, kk = e % d;
+        float s = acc[q];
+        for (int j = 0; j < MC; ++j) s = fmaf(p[t * MC + j], w2[kk * MC + j], s);
+        acc[q] = s;
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int e = tid + 256 * q;
+    if (e < nacc) {
+      const int t = e / d, kk = e % d;
+      if (t0 + t < T) O[(t0 + t) * ldo + (int64_t)h * d + kk] = acc[q];
+    }
+  }
+}
+
+}  // namespace ttt

@@ -1,0 +1,678 @@
+// C ABI of the large-chunk TTT layer (see include/ttt.h for the contract).
+//
+// Host side: argument validation, workspace carving, TMA tensor-map encoding
+// and the launch sequences of update / apply / chunked.  All device work runs
+// in the kernels of kernels_tc.cuh (bf16 tensor-core path) and
+// kernels_simt.cuh (memory-bound and fp32 paths); nothing here computes on
+// the CPU.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "kernels_simt.cuh"
+#include "kernels_tc.cuh"
+#include "ttt.h"
+
+using namespace ttt;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+// ---- per-kernel event timing (ttt_profile_*)
+struct ProfPair {
+  cudaEvent_t a, b;
+  int kind;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<ProfPair> g_prof_pending;
+std::vector<cudaEvent_t> g_prof_pool;
+double g_prof_ms[TTT_PROF_KINDS] = {0};
+uint64_t g_prof_n[TTT_PROF_KINDS] = {0};
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Records an event pair around the launches issued during its lifetime.
+struct ProfScope {
+  cudaEvent_t a = nullptr, b = nullptr;
+  cudaStream_t s;
+  int kind;
+  ProfScope(int k, cudaStream_t st) : s(st), kind(k) {
+    if (!g_prof_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    a = prof_event();
+    b = prof_event();
+    if (a && b) cudaEventRecord(a, s);
+  }
+  ~ProfScope() {
+    if (!a || !b) return;
+    cudaEventRecord(b, s);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_pending.push_back({a, b, kind});
+  }
+};
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+constexpr int kMaxSplits = 64;
+constexpr int kAssumedMaxSms = 160;
+
+struct Ws {
+  unsigned int* status;
+  __nv_bfloat16* wsh;  // [3][H*m][d]: W1, W3, W2^T
+  __nv_bfloat16* w2b;  // [H][d][m]
+  float* G;            // [3][H*m*d]
+  float* partial;      // [S_max][3][H*m*d]
+  float* X;            // [3H][m*d]
+  float* X2;           // [3H][m*d]
+  float* A;            // [3H][r*r]
+  float* B;            // [3H][r*r]
+  float* norms;        // [3H]
+  float* stepn;        // [2*3H]
+  float* rk;           // [T][H]
+  float* rq;           // [T][H]
+  size_t total;
+  int s_max;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int split_cap(const ttt_dims& d, ttt_dtype dt) {
+  const int slices = dt == TTT_BF16 ? d.heads * d.m / TC_MS : d.heads * d.m / F32_MS;
+  const int want = dt == TTT_BF16 ? kAssumedMaxSms / std::max(1, slices) : 2 * kAssumedMaxSms / std::max(1, slices);
+  return std::max(1, std::min(kMaxSplits, want));
+}
+
+bool dims_ok(const ttt_dims& d) { return d.heads >= 1 && d.d >= 1 && d.m >= 1 && d.heads <= 4096; }
+
+int dims_supported(const ttt_dims& d, ttt_dtype dt) {
+  if (dt == TTT_BF16) return (d.d == 128 || d.d == 192) && d.m % TC_MS == 0 ? TTT_OK : TTT_ERR_UNSUPPORTED;
+  if (dt == TTT_FP32) return (d.d <= 256 && d.d % 4 == 0 && d.m % F32_MS == 0) ? TTT_OK : TTT_ERR_UNSUPPORTED;
+  return TTT_ERR_INVALID;
+}
+
+Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
+  Ws w{};
+  const size_t H = dm.heads, d = dm.d, m = dm.m;
+  const size_t n = H * m * d;
+  const size_t r = std::min(d, m);
+  w.s_max = split_cap(dm, dt);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = up256(off + bytes);
+    return o;
+  };
+  const size_t o_status = take(256);
+  const size_t o_wsh = take(3 * n * 2);
+  const size_t o_w2b = take(n * 2);
+  const size_t o_G = take(3 * n * 4);
+  const size_t o_p = take((size_t)w.s_max * 3 * n * 4);
+  const size_t o_X = take(3 * n * 4);
+  const size_t o_X2 = take(3 * n * 4);
+  const size_t o_A = take(3 * H * r * r * 4);
+  const size_t o_B = take(3 * H * r * r * 4);
+  const size_t o_norms = take(3 * H * 4);
+  const size_t o_stepn = take(6 * H * 4);
+  const size_t o_rk = take((size_t)std::max<int64_t>(T, 1) * H * 4);
+  const size_t o_rq = take((size_t)std::max<int64_t>(T, 1) * H * 4);
+  w.total = off;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  if (b) {
+    w.status = reinterpret_cast<unsigned int*>(b + o_status);
+    w.wsh = reinterpret_cast<__nv_bfloat16*>(b + o_wsh);
+    w.w2b = reinterpret_cast<__nv_bfloat16*>(b + o_w2b);
+    w.G = reinterpret_cast<float*>(b + o_G);
+    w.partial = reinterpret_cast<float*>(b + o_p);
+    w.X = reinterpret_cast<float*>(b + o_X);
+    w.X2 = reinterpret_cast<float*>(b + o_X2);
+    w.A = reinterpret_cast<float*>(b + o_A);
+    w.B = reinterpret_cast<float*>(b + o_B);
+    w.norms = reinterpret_cast<float*>(b + o_norms);
+    w.stepn = reinterpret_cast<float*>(b + o_stepn);
+    w.rk = reinterpret_cast<float*>(b + o_rk);
+    w.rq = reinterpret_cast<float*>(b + o_rq);
+  }
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long v = [] {
+    const char* e = std::getenv("TTT_WAIT_TIMEOUT_MS");
+    if (e && *e) {
+      long long ms = std::atoll(e);
+      if (ms > 0) return (unsigned long long)ms * 1000000ull;
+    }
+    return kDefaultTimeoutNs;
+  }();
+  return v;
+}
+
+// ---- TMA tensor maps (driver entry point fetched once through the runtime)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] with row stride `row_bytes`, 128-byte swizzled boxes.
+bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+               uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+#define TTT_LAUNCHED()                                         \
+  do {                                                         \
+    g_launches.fetch_add(1, std::memory_order_relaxed);        \
+    if (cudaPeekAtLastError() != cudaSuccess) {                \
+      (void)cudaGetLastError();                                \
+      return TTT_ERR_CUDA;                                     \
+    }                                                          \
+  } while (0)
+
+#define TTT_CHECK(expr)                        \
+  do {                                         \
+    if ((expr) != cudaSuccess) {               \
+      (void)cudaGetLastError();                \
+      return TTT_ERR_CUDA;                     \
+    }                                          \
+  } while (0)
+
+#define TTT_TRY(expr)           \
+  do {                          \
+    int rc_ = (expr);           \
+    if (rc_ != TTT_OK) return rc_; \
+  } while (0)
+
+int grid1d(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(b, (int64_t)sm_count() * 32));
+}
+
+size_t esize(ttt_dtype dt) { return dt == TTT_BF16 ? 2 : 4; }
+
+int64_t eff_ld(int64_t ld, const ttt_dims& d) { return ld == 0 ? (int64_t)d.heads * d.d : ld; }
+
+int check_tokens(const void* p, int64_t ld, const ttt_dims& d, ttt_dtype dt, int64_t T) {
+  if (T == 0) return TTT_OK;
+  if (!p) return TTT_ERR_INVALID;
+  if (ld < (int64_t)d.heads * d.d) return TTT_ERR_INVALID;
+  if (!aligned16(p)) return TTT_ERR_ALIGN;
+  if ((ld * (int64_t)esize(dt)) % 16 != 0) return TTT_ERR_ALIGN;
+  return TTT_OK;
+}
+
+int check_common(const ttt_dims& dims, ttt_dtype dt, int64_t T, void* ws, size_t ws_bytes) {
+  if (dt != TTT_FP32 && dt != TTT_BF16) return TTT_ERR_INVALID;
+  if (!dims_ok(dims) || T < 0) return TTT_ERR_INVALID;
+  TTT_TRY(dims_supported(dims, dt));
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTT_ERR_WORKSPACE;
+  if (ws_bytes < carve(nullptr, dims, T, dt).total) return TTT_ERR_WORKSPACE;
+  return TTT_OK;
+}
+
+int check_weights(const ttt_weights& W) {
+  if (!W.W1 || !W.W3 || !W.W2) return TTT_ERR_INVALID;
+  if (!aligned16(W.W1) || !aligned16(W.W3) || !aligned16(W.W2)) return TTT_ERR_ALIGN;
+  return TTT_OK;
+}
+
+// ---- launch helpers
+
+template <typename T>
+int launch_rownorm(T* X, int64_t ld, int64_t rows, const ttt_dims& d, float* r_out, int mode, cudaStream_t s) {
+  if (rows == 0) return TTT_OK;
+  const int threads = 256;
+  const int64_t warps = rows;
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((warps * 32 + threads - 1) / threads,
+                                                                   (int64_t)sm_count() * 16));
+  ProfScope ps(TTT_PROF_NORM, s);
+  k_rownorm<T><<<blocks, threads, 0, s>>>(X, ld, rows, d.heads, d.d, r_out, mode);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+int launch_rownorm_any(const void* X, int64_t ld, int64_t rows, const ttt_dims& d, ttt_dtype dt, float* r_out,
+                       cudaStream_t s) {
+  if (dt == TTT_BF16)
+    return launch_rownorm<__nv_bfloat16>((__nv_bfloat16*)X, ld, rows, d, r_out, 0, s);
+  return launch_rownorm<float>((float*)X, ld, rows, d, r_out, 0, s);
+}
+
+int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStream_t s) {
+  const int64_t n = (int64_t)d.heads * d.m * d.d;
+  ProfScope ps(TTT_PROF_SHADOW, s);
+  k_shadow<<<grid1d(n, 256), 256, 0, s>>>(W.W1, W.W3, W.W2, w.wsh, w.w2b, d.heads, d.d, d.m);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+// gradient over T tokens -> G (fp32, [3][H*m*d]); shadow of W must be current (bf16)
+int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta,
+             const float* rk, int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, float* G, cudaStream_t s) {
+  const int64_t n = (int64_t)d.heads * d.m * d.d;
+  if (T == 0) {
+    TTT_CHECK(cudaMemsetAsync(G, 0, 3 * n * sizeof(float), s));
+    return TTT_OK;
+  }
+  int S = 1;
+  if (dt == TTT_BF16) {
+    const int tiles = (int)((T + TC_TILE - 1) / TC_TILE);
+    const int slices = d.m / TC_MS;
+    S = std::max(1, std::min({sm_count() / std::max(1, slices * d.heads), w.s_max, tiles}));
+    CUtensorMap tK, tV, tW;
+    const uint64_t hd = (uint64_t)d.heads * d.d;
+    if (!tmap_bf16(&tK, K, hd, (uint64_t)T, (uint64_t)ldk * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tV, V, hd, (uint64_t)T, (uint64_t)ldv * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tW, w.wsh, (uint64_t)d.d, 3ull * d.heads * d.m, (uint64_t)d.d * 2, 64, 64)) return TTT_ERR_CUDA;
+    dim3 grid(slices, d.heads, S);
+    ProfScope ps(TTT_PROF_GRAD, s);
+    if (d.d == 192) {
+      auto k = k_update_grad_tc<192>;
+      TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<192>::ALLOC));
+      k<<<grid, TC_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tW, eta, rk, w.partial, T, d.heads, d.m, tiles, S,
+                                                         w.status, wait_timeout_ns());
+    } else {
+      auto k = k_update_grad_tc<128>;
+      TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<128>::ALLOC));
+      k<<<grid, TC_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tW, eta, rk, w.partial, T, d.heads, d.m, tiles, S,
+                                                         w.status, wait_timeout_ns());
+    }
+    TTT_LAUNCHED();
+  } else {
+    const int tiles = (int)((T + F32_TT - 1) / F32_TT);
+    const int slices = d.m / F32_MS;
+    S = std::max(1, std::min({2 * sm_count() / std::max(1, slices * d.heads), w.s_max, tiles}));
+    const size_t smem =
+        (size_t)(3 * F32_MS * d.d + 2 * F32_TT * d.d + 3 * F32_TT * F32_MS + 2 * F32_TT) * sizeof(float);
+    TTT_CHECK(cudaFuncSetAttribute(k_grad_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    ProfScope ps(TTT_PROF_GRAD, s);
+    k_grad_f32<<<dim3(slices, d.heads, S), 256, smem, s>>>((const float*)K, ldk, (const float*)V, ldv, eta, rk, W.W1,
+                                                           W.W3, W.W2, w.partial, T, d.heads, d.d, d.m, S);
+    TTT_LAUNCHED();
+  }
+  ProfScope ps(TTT_PROF_REDUCE, s);
+  k_reduce_splits<<<grid1d(3 * n / 4, 256), 256, 0, s>>>(w.partial, S, 3 * n, G);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+// Newton-Schulz + weight step from G; refreshes the bf16 shadow in bf16 mode.
+int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const ttt_dims& d, const Ws& w,
+                cudaStream_t s) {
+  const int H = d.heads, mm = d.m, dd = d.d;
+  const int64_t n = (int64_t)mm * dd;
+  const int nb = 3 * H;
+  const int r = std::min(mm, dd), c = std::max(mm, dd);
+  const float* D = G;
+  int from_x = 0;
+  ProfScope ps(TTT_PROF_NS, s);
+  if (ns.iters > 0) {
+    k_frob_norms<<<nb, 256, 0, s>>>(G, n, w.norms);
+    TTT_LAUNCHED();
+    k_ns_init<<<dim3(grid1d(n, 256) / nb + 1, nb), 256, 0, s>>>(G, w.X, w.norms, H, dd, mm, ns.eps);
+    TTT_LAUNCHED();
+    float* X = w.X;
+    float* X2 = w.X2;
+    const int rt = (r + 63) / 64, ct = (c + 63) / 64;
+    for (int it = 0; it < ns.iters; ++it) {
+      k_gemm_f32<true><<<dim3(rt, rt, nb), 256, 0, s>>>(r, r, c, X, c, n, X, c, n, w.A, r, (int64_t)r * r, nullptr,
+                                                         1.f, 0.f);
+      TTT_LAUNCHED();
+      k_gemm_f32<false><<<dim3(rt, rt, nb), 256, 0, s>>>(r, r, r, w.A, r, (int64_t)r * r, w.A, r, (int64_t)r * r, w.B,
+                                                          r, (int64_t)r * r, w.A, ns.c, ns.b);
+      TTT_LAUNCHED();
+      k_gemm_f32<false><<<dim3(ct, rt, nb), 256, 0, s>>>(r, c, r, w.B, r, (int64_t)r * r, X, c, n, X2, c, n, X, 1.f,
+                                                          ns.a);
+      TTT_LAUNCHED();
+      std::swap(X, X2);
+    }
+    D = X;
+    from_x = 1;
+  }
+  k_step_norms<<<nb, 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, from_x, w.stepn);
+  TTT_LAUNCHED();
+  k_step_apply<<<dim3(grid1d(n, 256) / nb + 1, nb), 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, from_x,
+                                                                 ns.renorm, w.stepn);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+int run_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const ttt_dims& d, ttt_dtype dt, const Ws& w,
+             cudaStream_t s) {
+  TTT_TRY(run_ns_step(W, G, ns, d, w, s));
+  if (dt == TTT_BF16) TTT_TRY(launch_shadow(W, w, d, s));
+  return TTT_OK;
+}
+
+int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t ldo, const float* rq, int64_t T,
+              const ttt_dims& d, ttt_dtype dt, const Ws& w, cudaStream_t s) {
+  if (T == 0) return TTT_OK;
+  if (dt == TTT_BF16) {
+    const int tiles = (int)((T + TC_TILE - 1) / TC_TILE);
+    const int n_items = tiles * d.heads;
+    CUtensorMap tQ, tW, tW2;
+    const uint64_t hd = (uint64_t)d.heads * d.d;
+    if (!tmap_bf16(&tQ, Q, hd, (uint64_t)T, (uint64_t)ldq * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tW, w.wsh, (uint64_t)d.d, 3ull * d.heads * d.m, (uint64_t)d.d * 2, 64, 64)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tW2, w.w2b, (uint64_t)d.m, (uint64_t)d.heads * d.d, (uint64_t)d.m * 2, 64, (uint32_t)d.d))
+      return TTT_ERR_CUDA;
+    const int grid = std::min(n_items, sm_count());
+    ProfScope ps(TTT_PROF_APPLY, s);
+    if (d.d == 192) {
+      auto k = k_apply_tc<192>;
+      TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<192>::ALLOC));
+      k<<<grid, TC_THREADS, ApLayout<192>::ALLOC, s>>>(tQ, tW, tW2, rq, (__nv_bfloat16*)O, ldo, T, d.heads, d.m,
+                                                        n_items, w.status, wait_timeout_ns());
+    } else {
+      auto k = k_apply_tc<128>;
+      TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<128>::ALLOC));
+      k<<<grid, TC_THREADS, ApLayout<128>::ALLOC, s>>>(tQ, tW, tW2, rq, (__nv_bfloat16*)O, ldo, T, d.heads, d.m,
+                                                        n_items, w.status, wait_timeout_ns());
+    }
+    TTT_LAUNCHED();
+  } else {
+    const size_t smem = (size_t)(F32_TT * d.d + 2 * F32_MS * d.d + d.d * F32_MS + F32_TT * F32_MS + F32_TT) * 4;
+    TTT_CHECK(cudaFuncSetAttribute(k_apply_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    ProfScope ps(TTT_PROF_APPLY, s);
+    k_apply_f32<<<dim3((unsigned)((T + F32_TT - 1) / F32_TT), d.heads), 256, smem, s>>>(
+        (const float*)Q, ldq, rq, W.W1, W.W3, W.W2, (float*)O, ldo, T, d.heads, d.d, d.m);
+    TTT_LAUNCHED();
+  }
+  return TTT_OK;
+}
+
+int check_ns(const ttt_ns_cfg* ns) {
+  if (!ns || ns->iters < 0 || ns->iters > 64 || !(ns->eps >= 0.f)) return TTT_ERR_INVALID;
+  return TTT_OK;
+}
+
+const ttt_io_cfg kDefaultIo = {1, 0, 0, 0, 0};
+
+}  // namespace
+
+extern "C" {
+
+size_t ttt_workspace_bytes(ttt_dims dims, int64_t T, ttt_dtype dtype) {
+  if (!dims_ok(dims) || T < 0 || (dtype != TTT_FP32 && dtype != TTT_BF16)) return 0;
+  return carve(nullptr, dims, T, dtype).total;
+}
+
+int ttt_reset_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 256) return TTT_ERR_WORKSPACE;
+  TTT_CHECK(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream));
+  return TTT_OK;
+}
+
+int ttt_poll_status(const void* ws, void* stream) {
+  if (!ws) return TTT_ERR_WORKSPACE;
+  TTT_CHECK(cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned int v = 0;
+  TTT_CHECK(cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost));
+  return v == DEV_OK ? TTT_OK : TTT_ERR_TIMEOUT;
+}
+
+int ttt_l2norm(void* X, int64_t T, ttt_dims dims, int64_t ld, ttt_dtype dtype, void* stream) {
+  if ((dtype != TTT_FP32 && dtype != TTT_BF16) || !dims_ok(dims) || T < 0) return TTT_ERR_INVALID;
+  if (dims.d % (dtype == TTT_BF16 ? 8 : 4)) return TTT_ERR_UNSUPPORTED;
+  ld = eff_ld(ld, dims);
+  TTT_TRY(check_tokens(X, ld, dims, dtype, T));
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == TTT_BF16) return launch_rownorm<__nv_bfloat16>((__nv_bfloat16*)X, ld, T, dims, nullptr, 1, s);
+  return launch_rownorm<float>((float*)X, ld, T, dims, nullptr, 1, s);
+}
+
+int ttt_shortconv2d(const void* V, int64_t ld_v, void* Vout, int64_t ld_out, const float* taps, int N, int h, int w,
+                    int C, int act, ttt_dtype dtype, void* stream) {
+  if (dtype != TTT_FP32 && dtype != TTT_BF16) return TTT_ERR_INVALID;
+  if (N < 0 || h < 1 || w < 1 || C < 1 || (act != 0 && act != 1)) return TTT_ERR_INVALID;
+  if (C % 8) return TTT_ERR_UNSUPPORTED;
+  if (ld_v == 0) ld_v = C;
+  if (ld_out == 0) ld_out = C;
+  if (ld_v < C || ld_out < C) return TTT_ERR_INVALID;
+  if (N == 0) return TTT_OK;
+  if (!V || !Vout || !taps || V == Vout) return TTT_ERR_INVALID;
+  if (!aligned16(V) || !aligned16(Vout) || (ld_v * (int64_t)esize(dtype)) % 16 || (ld_out * (int64_t)esize(dtype)) % 16)
+    return TTT_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t ntok = (int64_t)N * h * w;
+  const int vn = dtype == TTT_BF16 ? 8 : 4;
+  const int nvec = C / vn;
+  dim3 block(std::min(nvec, 128), std::max(1, 256 / std::min(nvec, 128)));
+  dim3 grid((nvec + block.x - 1) / block.x,
+            (unsigned)std::max<int64_t>(1, std::min<int64_t>((ntok + block.y - 1) / block.y, 65535)));
+  ProfScope ps(TTT_PROF_CONV, s);
+  if (dtype == TTT_BF16)
+    k_shortconv<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)V, ld_v, (__nv_bfloat16*)Vout, ld_out,
+                                                      taps, N, h, w, C, act);
+  else
+    k_shortconv<float><<<grid, block, 0, s>>>((const float*)V, ld_v, (float*)Vout, ld_out, taps, N, h, w, C, act);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, ttt_dims dims,
+             const ttt_io_cfg* io, ttt_dtype dtype, float* G, void* ws, size_t ws_bytes, void* stream) {
+  TTT_TRY(check_common(dims, dtype, T, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  if (!io) io = &kDefaultIo;
+  const int64_t ldk = eff_ld(io->ld_k, dims), ldv = eff_ld(io->ld_v, dims);
+  TTT_TRY(check_tokens(K, ldk, dims, dtype, T));
+  TTT_TRY(check_tokens(V, ldv, dims, dtype, T));
+  if (!G) return TTT_ERR_INVALID;
+  if (!aligned16(G)) return TTT_ERR_ALIGN;
+  if (T > 0 && !eta) return TTT_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  Ws w = carve(ws, dims, T, dtype);
+  const float* rk = nullptr;
+  if (io->qk_l2norm && T > 0) {
+    TTT_TRY(launch_rownorm_any(K, ldk, T, dims, dtype, w.rk, s));
+    rk = w.rk;
+  }
+  if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
+  return run_grad(W, K, ldk, V, ldv, eta, rk, T, dims, dtype, w, G, s);
+}
+
+int ttt_step(ttt_weights W, const float* G, const ttt_ns_cfg* ns, ttt_dims dims, ttt_dtype dtype, void* ws,
+             size_t ws_bytes, void* stream) {
+  TTT_TRY(check_common(dims, dtype, 0, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  TTT_TRY(check_ns(ns));
+  if (!G) return TTT_ERR_INVALID;
+  Ws w = carve(ws, dims, 0, dtype);
+  return run_step(W, G, *ns, dims, dtype, w, (cudaStream_t)stream);
+}
+
+int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, int steps,
+               const ttt_ns_cfg* ns, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes,
+               void* stream) {
+  TTT_TRY(check_common(dims, dtype, T, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  TTT_TRY(check_ns(ns));
+  if (steps < 0) return TTT_ERR_INVALID;
+  if (!io) io = &kDefaultIo;
+  const int64_t ldk = eff_ld(io->ld_k, dims), ldv = eff_ld(io->ld_v, dims);
+  TTT_TRY(check_tokens(K, ldk, dims, dtype, T));
+  TTT_TRY(check_tokens(V, ldv, dims, dtype, T));
+  if (T > 0 && !eta) return TTT_ERR_INVALID;
+  if (T == 0 || steps == 0) return TTT_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  Ws w = carve(ws, dims, T, dtype);
+  const float* rk = nullptr;
+  if (io->qk_l2norm) {
+    TTT_TRY(launch_rownorm_any(K, ldk, T, dims, dtype, w.rk, s));
+    rk = w.rk;
+  }
+  if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
+  for (int st = 0; st < steps; ++st) {
+    TTT_TRY(run_grad(W, K, ldk, V, ldv, eta, rk, T, dims, dtype, w, w.G, s));
+    TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+  }
+  return TTT_OK;
+}
+
+int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype,
+              void* ws, size_t ws_bytes, void* stream) {
+  TTT_TRY(check_common(dims, dtype, T, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  if (!io) io = &kDefaultIo;
+  const int64_t ldq = eff_ld(io->ld_q, dims), ldo = eff_ld(io->ld_o, dims);
+  TTT_TRY(check_tokens(Q, ldq, dims, dtype, T));
+  TTT_TRY(check_tokens(O, ldo, dims, dtype, T));
+  if (T > 0 && Q == O) return TTT_ERR_INVALID;
+  if (T == 0) return TTT_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  Ws w = carve(ws, dims, T, dtype);
+  const float* rq = nullptr;
+  if (io->qk_l2norm) {
+    TTT_TRY(launch_rownorm_any(Q, ldq, T, dims, dtype, w.rq, s));
+    rq = w.rq;
+  }
+  if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
+  return run_apply(W, Q, ldq, O, ldo, rq, T, dims, dtype, w, s);
+}
+
+int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, const float* eta, void* O, int64_t T,
+                int64_t chunk, int order, int steps, const ttt_ns_cfg* ns, ttt_dims dims, const ttt_io_cfg* io,
+                ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (chunk <= 0 || (order != 0 && order != 1) || steps < 0) return TTT_ERR_INVALID;
+  const int64_t cmax = std::min<int64_t>(chunk, std::max<int64_t>(T, 0));
+  TTT_TRY(check_common(dims, dtype, cmax, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  TTT_TRY(check_ns(ns));
+  if (!io) io = &kDefaultIo;
+  const int64_t ldq = eff_ld(io->ld_q, dims), ldk = eff_ld(io->ld_k, dims);
+  const int64_t ldv = eff_ld(io->ld_v, dims), ldo = eff_ld(io->ld_o, dims);
+  TTT_TRY(check_tokens(Q, ldq, dims, dtype, T));
+  TTT_TRY(check_tokens(K, ldk, dims, dtype, T));
+  TTT_TRY(check_tokens(V, ldv, dims, dtype, T));
+  TTT_TRY(check_tokens(O, ldo, dims, dtype, T));
+  if (T > 0 && (!eta || Q == O)) return TTT_ERR_INVALID;
+  if (T == 0) return TTT_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  Ws w = carve(ws, dims, cmax, dtype);
+  const size_t es = esize(dtype);
+  if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
+  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+    const int64_t tc = std::min(chunk, T - c0);
+    const uint8_t* q = static_cast<const uint8_t*>(Q) + c0 * ldq * es;
+    const uint8_t* k = static_cast<const uint8_t*>(K) + c0 * ldk * es;
+    const uint8_t* v = static_cast<const uint8_t*>(V) + c0 * ldv * es;
+    uint8_t* o = static_cast<uint8_t*>(O) + c0 * ldo * es;
+    const float* e = eta + c0 * dims.heads;
+    const float* rk = nullptr;
+    const float* rq = nullptr;
+    if (io->qk_l2norm) {
+      TTT_TRY(launch_rownorm_any(k, ldk, tc, dims, dtype, w.rk, s));
+      TTT_TRY(launch_rownorm_any(q, ldq, tc, dims, dtype, w.rq, s));
+      rk = w.rk;
+      rq = w.rq;
+    }
+    if (order == 0) TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
+    for (int st = 0; st < steps; ++st) {
+      TTT_TRY(run_grad(W, k, ldk, v, ldv, e, rk, tc, dims, dtype, w, w.G, s));
+      TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+    }
+    if (order == 1) TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
+  }
+  return TTT_OK;
+}
+
+const char* ttt_status_string(int status) {
+  switch (status) {
+    case TTT_OK: return "ok";
+    case TTT_ERR_INVALID: return "invalid argument";
+    case TTT_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case TTT_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case TTT_ERR_CUDA: return "CUDA runtime error or failed launch";
+    case TTT_ERR_TIMEOUT: return "device-side wait timed out";
+    case TTT_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+uint64_t ttt_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ttt_profile_enable(int on) {
+  g_prof_on.store(on != 0);
+  return TTT_OK;
+}
+
+int ttt_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& p : g_prof_pending) {
+    cudaEventSynchronize(p.b);
+    g_prof_pool.push_back(p.a);
+    g_prof_pool.push_back(p.b);
+  }
+  g_prof_pending.clear();
+  for (int k = 0; k < TTT_PROF_KINDS; ++k) {
+    g_prof_ms[k] = 0;
+    g_prof_n[k] = 0;
+  }
+  return TTT_OK;
+}
+
+int ttt_profile_query(int kind, double* total_ms, uint64_t* count) {
+  if (kind < 0 || kind >= TTT_PROF_KINDS) return TTT_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& p : g_prof_pending) {
+    if (cudaEventSynchronize(p.b) != cudaSuccess) return TTT_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, p.a, p.b) != cudaSuccess) return TTT_ERR_CUDA;
+    g_prof_ms[p.kind] += ms;
+    g_prof_n[p.kind] += 1;
+    g_prof_pool.push_back(p.a);
+    g_prof_pool.push_back(p.b);
+  }
+  g_prof_pending.clear();
+  if (total_ms) *total_ms = g_prof_ms[kind];
+  if (count) *count = g_prof_n[kind];
+  return TTT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,177 @@
+"""GPU parity of each entry point against the fp64 oracle at small sizes
+(several 128-token tiles plus a ragged tail), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from test_weight_layers_b200 import ttt as T
+
+from _gpu import (TOL_BF16, TOL_FP32, DevWeights, check_status, f64, need_gpu, rand_eta, rand_tokens, rand_weights,
+                  rel_fro, weight_errors)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_l2norm_in_place(dtype):
+    H, d, T_ = 4, 192, 333
+    X = rand_tokens(T_, H, d, dtype, 1, ld=H * d + 8, scale=3.0)
+    X[5, :d] = 0  # zero row stays zero (eps clamp)
+    ref = O.l2norm_heads(f64(X), H, d)
+    Xd = X.cuda()
+    T.ttt_l2norm(Xd, T_, T.dims(H, d, 64), ld=H * d + 8)
+    torch.cuda.synchronize()
+    got = f64(Xd)
+    tol = 4e-3 if dtype == torch.bfloat16 else 1e-6
+    assert rel_fro(got[:, :H * d], ref) < tol
+    assert np.all(got[5, :d] == 0)
+    assert np.array_equal(got[:, H * d:], f64(X)[:, H * d:])  # padding untouched
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("act", [0, 1])
+def test_shortconv2d(dtype, act):
+    N, h, w, C = 3, 5, 7, 64
+    V = rand_tokens(N * h * w, 1, C, dtype, 2, ld=C + 8)
+    taps = torch.randn((C, 3, 3), generator=torch.Generator().manual_seed(3)) / 3
+    ref = O.shortconv2d(f64(V)[:, :C], taps.double().numpy(), N, h, w, act)
+    out = torch.zeros((N * h * w, C), dtype=dtype, device="cuda")
+    T.ttt_shortconv2d(V.cuda(), out, taps.cuda(), N, h, w, C, act, ld_v=C + 8, ld_out=C)
+    torch.cuda.synchronize()
+    tol = 5e-3 if dtype == torch.bfloat16 else 1e-6
+    assert rel_fro(f64(out), ref) < tol
+
+
+@pytest.mark.parametrize("H,d,m,T_", [(1, 192, 64, 1), (2, 192, 768, 300), (3, 128, 192, 1000), (4, 192, 256, 129)])
+def test_apply_bf16(H, d, m, T_):
+    W = DevWeights(*rand_weights(H, d, m, 10 + m))
+    Q = rand_tokens(T_, H, d, torch.bfloat16, 11)
+    dm = T.dims(H, d, m)
+    ws = T.workspace(dm, T_, T.TTT_BF16)
+    O_ = torch.full((T_, H * d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    T.ttt_apply(W.abi, Q.cuda(), O_, T_, dm, T.io_cfg(), ws)
+    check_status(ws)
+    ref = O.apply(W.oracle(), f64(Q))
+    err = rel_fro(f64(O_), ref)
+    assert err < 1e-2, err
+
+
+def test_apply_bf16_strided_rows():
+    H, d, m, T_ = 2, 192, 128, 260
+    W = DevWeights(*rand_weights(H, d, m, 12))
+    Q = rand_tokens(T_, H, d, torch.bfloat16, 13, ld=H * d + 64)
+    dm = T.dims(H, d, m)
+    ws = T.workspace(dm, T_, T.TTT_BF16)
+    O_ = torch.zeros((T_, H * d + 16), dtype=torch.bfloat16, device="cuda")
+    T.ttt_apply(W.abi, Q.cuda(), O_, T_, dm, T.io_cfg(ld_q=H * d + 64, ld_o=H * d + 16), ws)
+    check_status(ws)
+    ref = O.apply(W.oracle(), f64(Q)[:, :H * d])
+    assert rel_fro(f64(O_)[:, :H * d], ref) < 1e-2
+    assert torch.all(O_[:, H * d:] == 0)
+
+
+@pytest.mark.parametrize("qk", [1, 0])
+def test_apply_fp32(qk):
+    H, d, m, T_ = 2, 64, 128, 77
+    W = DevWeights(*rand_weights(H, d, m, 14))
+    Q = rand_tokens(T_, H, d, torch.float32, 15)
+    dm = T.dims(H, d, m)
+    ws = T.workspace(dm, T_, T.TTT_FP32)
+    O_ = torch.zeros((T_, H * d), dtype=torch.float32, device="cuda")
+    T.ttt_apply(W.abi, Q.cuda(), O_, T_, dm, T.io_cfg(qk_l2norm=qk), ws)
+    check_status(ws)
+    ref = O.apply(W.oracle(), f64(Q), qk_l2norm=bool(qk))
+    assert rel_fro(f64(O_), ref) < 1e-5
+
+
+def _grad_case(H, d, m, T_, dtype, seed=20):
+    W = DevWeights(*rand_weights(H, d, m, seed))
+    K = rand_tokens(T_, H, d, dtype, seed + 1)
+    V = rand_tokens(T_, H, d, dtype, seed + 2)
+    eta = rand_eta(T_, H, seed + 3, scale=1.0)
+    return W, K, V, eta
+
+
+def _run_grad(W, K, V, eta, dm, dtype_code):
+    T_ = K.shape[0]
+    ws = T.workspace(dm, T_, dtype_code)
+    n = dm.heads * dm.m * dm.d
+    G = torch.full((3 * n,), float("nan"), dtype=torch.float32, device="cuda")
+    T.ttt_grad(W.abi, K.cuda(), V.cuda(), eta.cuda(), T_, dm, T.io_cfg(), G, ws)
+    check_status(ws)
+    H, d, m = dm.heads, dm.d, dm.m
+    g = f64(G)
+    return O.FastWeights(g[:n].reshape(H, m, d), g[n:2 * n].reshape(H, m, d), g[2 * n:].reshape(H, d, m)), G
+
+
+@pytest.mark.parametrize("H,d,m,T_", [(1, 192, 64, 1), (2, 192, 128, 1000), (2, 128, 256, 129), (4, 192, 768, 384)])
+def test_grad_bf16(H, d, m, T_):
+    W, K, V, eta = _grad_case(H, d, m, T_, torch.bfloat16)
+    got, _ = _run_grad(W, K, V, eta, T.dims(H, d, m), T.TTT_BF16)
+    ref = O.grad(W.oracle(), O.l2norm_heads(f64(K), H, d), f64(V), f64(eta))
+    errs = weight_errors(got, ref)
+    assert max(errs) < 2e-2, errs
+
+
+@pytest.mark.parametrize("H,d,m,T_", [(1, 64, 128, 128), (2, 64, 64, 200), (1, 96, 32, 33)])
+def test_grad_fp32(H, d, m, T_):
+    W, K, V, eta = _grad_case(H, d, m, T_, torch.float32)
+    got, _ = _run_grad(W, K, V, eta, T.dims(H, d, m), T.TTT_FP32)
+    ref = O.grad(W.oracle(), O.l2norm_heads(f64(K), H, d), f64(V), f64(eta))
+    errs = weight_errors(got, ref)
+    assert max(errs) < 1e-5, errs
+
+
+@pytest.mark.parametrize("dt", [T.TTT_BF16, T.TTT_FP32])
+def test_grad_is_deterministic(dt):
+    dtype = torch.bfloat16 if dt == T.TTT_BF16 else torch.float32
+    d = 192 if dt == T.TTT_BF16 else 64
+    W, K, V, eta = _grad_case(2, d, 128, 1500, dtype, seed=30)
+    _, G1 = _run_grad(W, K, V, eta, T.dims(2, d, 128), dt)
+    _, G2 = _run_grad(W, K, V, eta, T.dims(2, d, 128), dt)
+    assert torch.equal(G1, G2)
+
+
+@pytest.mark.parametrize("dt,d,m", [(T.TTT_BF16, 192, 768), (T.TTT_BF16, 128, 64), (T.TTT_FP32, 64, 128),
+                                    (T.TTT_FP32, 96, 32)])
+@pytest.mark.parametrize("iters,renorm,lr", [(5, 1, 1.0), (0, 0, 0.01), (3, 0, 0.5)])
+def test_step_matches_oracle(dt, d, m, iters, renorm, lr):
+    H = 2
+    W = DevWeights(*rand_weights(H, d, m, 40))
+    Wo = W.oracle()
+    dtype = torch.bfloat16 if dt == T.TTT_BF16 else torch.float32
+    K = rand_tokens(64, H, d, torch.float32, 41)
+    V = rand_tokens(64, H, d, torch.float32, 42)
+    G = O.grad(Wo, O.l2norm_heads(f64(K), H, d), f64(V), f64(rand_eta(64, H, 43, 1.0)))
+    Gflat = torch.from_numpy(np.concatenate([G.W1.ravel(), G.W3.ravel(), G.W2.ravel()])).float()
+    dm = T.dims(H, d, m)
+    ws = T.workspace(dm, 0, dt)
+    cfg = O.NSConfig(iters=iters, renorm=renorm, lr=lr)
+    T.ttt_step(W.abi, Gflat.cuda(), T.ns_cfg(iters=iters, renorm=renorm, lr=lr), dm, dt, ws)
+    check_status(ws)
+    ref = O.muon_step(Wo, O.FastWeights(*(f64(x) for x in (Gflat[:H * m * d].reshape(H, m, d),
+                                                            Gflat[H * m * d:2 * H * m * d].reshape(H, m, d),
+                                                            Gflat[2 * H * m * d:].reshape(H, d, m)))), cfg)
+    errs = weight_errors(W.oracle(), ref)
+    assert max(errs) < 1e-5, errs
+    del dtype
+
+
+def test_update_eta_zero_keeps_weights_bf16():
+    H, d, m, T_ = 2, 192, 128, 500
+    W = DevWeights(*rand_weights(H, d, m, 50))
+    before = W.oracle()
+    K = rand_tokens(T_, H, d, torch.bfloat16, 51).cuda()
+    V = rand_tokens(T_, H, d, torch.bfloat16, 52).cuda()
+    eta = torch.zeros((T_, H), dtype=torch.float32, device="cuda")
+    dm = T.dims(H, d, m)
+    ws = T.workspace(dm, T_, T.TTT_BF16)
+    T.ttt_update(W.abi, K, V, eta, T_, 1, T.ns_cfg(), dm, T.io_cfg(), ws)
+    check_status(ws)
+    assert max(weight_errors(W.oracle(), before)) < 1e-6
