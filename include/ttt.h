@@ -59,7 +59,8 @@ typedef enum {
   TTT_ERR_WORKSPACE = -3,    /* workspace missing or smaller than ttt_workspace_bytes() */
   TTT_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
   TTT_ERR_TIMEOUT = -5,      /* a device-side wait gave up (reported through ttt_poll_status) */
-  TTT_ERR_ALIGN = -6         /* pointer or row stride violates the 16-byte alignment rule */
+  TTT_ERR_ALIGN = -6,        /* pointer or row stride violates the 16-byte alignment rule */
+  TTT_ERR_SCRATCH = -7       /* problem too large for the fixed scratch of ttt_apply_noalloc */
 } ttt_status;
 
 typedef enum { TTT_FP32 = 0, TTT_BF16 = 1 } ttt_dtype;
@@ -128,6 +129,35 @@ int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, in
 /* Apply: O[i] = f_W(q_i) for T query rows (Q and O may not alias). */
 int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
               const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* Apply without a workspace and without any allocation (no counterpart in the
+ * pages: this is a deployment convenience).  Computes exactly what ttt_apply
+ * computes, for callers that cannot hand the library device memory for scratch:
+ * hosts whose memory is fully reserved up front (a pool or arena that the
+ * library cannot draw from), plugin environments that forbid cudaMalloc and
+ * cudaFree, and latency-critical query loops that must not call into the
+ * allocator at all.  Its scratch (the bf16 copies of W, the per-token Q norms
+ * and a status word) lives in one fixed array of TTT_NOALLOC_SCRATCH_BYTES
+ * (8 MiB) that the library declares statically in device memory, so every GPU
+ * that loads the library holds those 8 MiB until the process exits.
+ *  - Limit: 8 * H * m * d bytes of weight copies plus at least 128 tokens of
+ *    norms (4 * H bytes each) must fit; larger dims return TTT_ERR_SCRATCH.
+ *    T itself is unbounded: the call walks the queries in token chunks sized
+ *    to the space left.  For 4 heads, d = 192, m = 768 that is 4.7 MiB of
+ *    weights and chunks of up to ~200k tokens.
+ *  - The first call on each device looks up that device's address of the
+ *    array (a host-side lookup, no allocation); make the first call on a device
+ *    before capturing a stream on it.
+ *  - Every call reuses the same array and leaves its contents behind; the call
+ *    clears the status word itself.  Calls whose work overlaps on the GPU (on
+ *    different streams, or from different host threads) race on the array:
+ *    order them on one stream.
+ *  - A device-side wait that times out cannot be polled here (there is no
+ *    workspace); O is then undefined.
+ * Arguments and layouts as for ttt_apply, minus the workspace. */
+#define TTT_NOALLOC_SCRATCH_BYTES (8u << 20)
+int ttt_apply_noalloc(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
+                      const ttt_io_cfg* io, ttt_dtype dtype, void* stream);
 
 /* Causal chunk carry over T tokens in chunks of `chunk` (the last may be shorter).
  * order 0: O_c = f_{W_(c-1)}(Q_c), then W_c = TTTUpdate(W_(c-1); chunk c);

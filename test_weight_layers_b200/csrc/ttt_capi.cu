@@ -433,6 +433,30 @@ int check_ns(const ttt_ns_cfg* ns) {
 
 const ttt_io_cfg kDefaultIo = {1, 0, 0, 0, 0};
 
+// ---- scratch of ttt_apply_noalloc: one fixed array in device memory, no allocation.
+// Host code only ever holds its per-device address from cudaGetSymbolAddress;
+// the symbol itself names a host-side shadow and is never passed to a kernel.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TTT_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device (looked up once per device).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  TTT_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return TTT_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    TTT_CHECK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    if (!p) return TTT_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return TTT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -576,6 +600,51 @@ int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims, c
   return run_apply(W, Q, ldq, O, ldo, rq, T, dims, dtype, w, s);
 }
 
+int ttt_apply_noalloc(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims, const ttt_io_cfg* io,
+                      ttt_dtype dtype, void* stream) {
+  if (dtype != TTT_FP32 && dtype != TTT_BF16) return TTT_ERR_INVALID;
+  if (!dims_ok(dims) || T < 0) return TTT_ERR_INVALID;
+  TTT_TRY(dims_supported(dims, dtype));
+  TTT_TRY(check_weights(W));
+  if (!io) io = &kDefaultIo;
+  const int64_t ldq = eff_ld(io->ld_q, dims), ldo = eff_ld(io->ld_o, dims);
+  TTT_TRY(check_tokens(Q, ldq, dims, dtype, T));
+  TTT_TRY(check_tokens(O, ldo, dims, dtype, T));
+  if (T > 0 && Q == O) return TTT_ERR_INVALID;
+  // scratch plan: [status 256 B | W1,W3,W2^T bf16 | W2 bf16 | per-token inverse norms of one token chunk]
+  const size_t n = (size_t)dims.heads * dims.m * dims.d;
+  const size_t fixed = 256 + up256(3 * n * 2) + up256(n * 2);
+  if (fixed >= TTT_NOALLOC_SCRATCH_BYTES) return TTT_ERR_SCRATCH;
+  const int64_t per_tok = (int64_t)dims.heads * 4;
+  const int64_t chunk = ((int64_t)(TTT_NOALLOC_SCRATCH_BYTES - fixed) / per_tok) / TC_TILE * TC_TILE;
+  if (chunk < TC_TILE) return TTT_ERR_SCRATCH;
+  if (T == 0) return TTT_OK;
+  void* base = nullptr;
+  TTT_TRY(noalloc_scratch(&base));
+  uint8_t* b = static_cast<uint8_t*>(base);
+  Ws w{};
+  w.status = reinterpret_cast<unsigned int*>(b);
+  w.wsh = reinterpret_cast<__nv_bfloat16*>(b + 256);
+  w.w2b = reinterpret_cast<__nv_bfloat16*>(b + 256 + up256(3 * n * 2));
+  float* rq_buf = reinterpret_cast<float*>(b + fixed);
+  cudaStream_t s = (cudaStream_t)stream;
+  TTT_CHECK(cudaMemsetAsync(w.status, 0, 256, s));
+  if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
+  const size_t es = esize(dtype);
+  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+    const int64_t tc = std::min(chunk, T - c0);
+    const uint8_t* q = static_cast<const uint8_t*>(Q) + c0 * ldq * es;
+    uint8_t* o = static_cast<uint8_t*>(O) + c0 * ldo * es;
+    const float* rq = nullptr;
+    if (io->qk_l2norm) {
+      TTT_TRY(launch_rownorm_any(q, ldq, tc, dims, dtype, rq_buf, s));
+      rq = rq_buf;
+    }
+    TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
+  }
+  return TTT_OK;
+}
+
 int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, const float* eta, void* O, int64_t T,
                 int64_t chunk, int order, int steps, const ttt_ns_cfg* ns, ttt_dims dims, const ttt_io_cfg* io,
                 ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream) {
@@ -631,6 +700,7 @@ const char* ttt_status_string(int status) {
     case TTT_ERR_CUDA: return "CUDA runtime error or failed launch";
     case TTT_ERR_TIMEOUT: return "device-side wait timed out";
     case TTT_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
+    case TTT_ERR_SCRATCH: return "problem too large for the fixed 8 MiB scratch of ttt_apply_noalloc";
     default: return "unknown status";
   }
 }

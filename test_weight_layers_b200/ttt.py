@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libttt.so")
 
 TTT_OK, TTT_ERR_INVALID, TTT_ERR_UNSUPPORTED, TTT_ERR_WORKSPACE = 0, -1, -2, -3
-TTT_ERR_CUDA, TTT_ERR_TIMEOUT, TTT_ERR_ALIGN = -4, -5, -6
+TTT_ERR_CUDA, TTT_ERR_TIMEOUT, TTT_ERR_ALIGN, TTT_ERR_SCRATCH = -4, -5, -6, -7
 TTT_FP32, TTT_BF16 = 0, 1
 
 
@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "ttt_update": (I, [Weights, P, P, P, I64, I, ctypes.POINTER(NSCfg), Dims, ctypes.POINTER(IOCfg), I, P, SZ,
                                P]),
             "ttt_apply": (I, [Weights, P, P, I64, Dims, ctypes.POINTER(IOCfg), I, P, SZ, P]),
+            "ttt_apply_noalloc": (I, [Weights, P, P, I64, Dims, ctypes.POINTER(IOCfg), I, P]),
             "ttt_chunked": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), Dims,
                                 ctypes.POINTER(IOCfg), I, P, SZ, P]),
             "ttt_status_string": (ctypes.c_char_p, [I]),
@@ -172,6 +173,12 @@ def ttt_update(W: Weights, K, V, eta, T, steps, ns: NSCfg, dm: Dims, io: IOCfg, 
 def ttt_apply(W: Weights, Q, O, T, dm: Dims, io: IOCfg, ws, stream=None):
     _check("ttt_apply", lib().ttt_apply(W, _ptr(Q), _ptr(O), T, dm, ctypes.byref(io), dtype_code(Q.dtype), _ptr(ws),
                                         ws.numel(), _stream(stream)))
+
+
+def ttt_apply_noalloc(W: Weights, Q, O, T, dm: Dims, io: IOCfg, stream=None):
+    """ttt_apply without a workspace: the library uses its own fixed 8 MiB device array as scratch."""
+    _check("ttt_apply_noalloc", lib().ttt_apply_noalloc(W, _ptr(Q), _ptr(O), T, dm, ctypes.byref(io),
+                                                        dtype_code(Q.dtype), _stream(stream)))
 
 
 def ttt_chunked(W: Weights, Q, K, V, eta, O, T, chunk, order, steps, ns: NSCfg, dm: Dims, io: IOCfg, ws, stream=None):
