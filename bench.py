@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="zipmap")
+    ap.add_argument("--frames", type=int, default=0, help="override the workload's frame count (profiling runs)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -444,6 +445,8 @@ def main():
     args = parse()
     from test_weight_layers_b200 import synth as S
     cfg = S.WORKLOADS[args.workload]
+    if args.frames:
+        cfg = cfg.with_frames(args.frames)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

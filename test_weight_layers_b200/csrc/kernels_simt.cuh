@@ -54,83 +54,171 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ---------------------------------------------------------------------------
 // L2 norms of (token, head) rows (VGG-T3 key design 1): one warp per token.
 // mode 0: write r[t*H + h] = 1 / max(||x||, 1e-12);  mode 1: scale X in place.
+// The whole row (H*d <= 128 16-byte vectors) is loaded before any reduction so
+// every lane has its loads in flight together; per-head sums are warp
+// reductions of lane partials masked by head.
+
+constexpr int RN_MAX_VEC = 4;  // 16-byte vectors per lane: H*d <= 128 * VN elements
 
 template <typename T>
-__global__ void k_rownorm(T* X, int64_t ld, int64_t rows, int H, int d, float* r_out, int mode) {
+__global__ void __launch_bounds__(256, 4) k_rownorm(T* X, int64_t ld, int64_t rows, int H, int d, float* r_out, int mode) {
   constexpr int VN = Vec16<T>::N;
   const int lane = threadIdx.x & 31;
   const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int nv = d / VN;
-  for (int64_t t = warp_id; t < rows; t += nwarps) {
-    T* row = X + t * ld;
-    for (int h = 0; h < H; ++h) {
-      float ss = 0.f;
-      for (int v = lane; v < nv; v += 32) {
-        float x[VN];
-        load16(row + h * d + v * VN, x);
-#pragma unroll
-        for (int i = 0; i < VN; ++i) ss = fmaf(x[i], x[i], ss);
-      }
-      ss = warp_sum(ss);
-      const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-      if (mode == 0) {
-        if (lane == 0) r_out[t * H + h] = inv;
-      } else {
+  const int nvt = H * d / VN;  // vectors per row
+  if (nvt > 32 * RN_MAX_VEC) {
+    // wide rows: one head at a time
+    const int nv = d / VN;
+    for (int64_t t = warp_id; t < rows; t += nwarps) {
+      T* row = X + t * ld;
+      for (int h = 0; h < H; ++h) {
+        float ss = 0.f;
         for (int v = lane; v < nv; v += 32) {
           float x[VN];
           load16(row + h * d + v * VN, x);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) x[i] *= inv;
-          store16(row + h * d + v * VN, x);
+          for (int i = 0; i < VN; ++i) ss = fmaf(x[i], x[i], ss);
+        }
+        ss = warp_sum(ss);
+        const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+        if (mode == 0) {
+          if (lane == 0) r_out[t * H + h] = inv;
+        } else {
+          for (int v = lane; v < nv; v += 32) {
+            float x[VN];
+            load16(row + h * d + v * VN, x);
+#pragma unroll
+            for (int i = 0; i < VN; ++i) x[i] *= inv;
+            store16(row + h * d + v * VN, x);
+          }
         }
       }
+    }
+    return;
+  }
+  for (int64_t t = warp_id; t < rows; t += nwarps) {
+    T* row = X + t * ld;
+    float x[RN_MAX_VEC][VN];
+    float ss[RN_MAX_VEC];
+    int hv[RN_MAX_VEC];
+#pragma unroll
+    for (int k = 0; k < RN_MAX_VEC; ++k) {
+      const int v = lane + 32 * k;
+      hv[k] = -1;
+      ss[k] = 0.f;
+      if (v < nvt) {
+        load16(row + v * VN, x[k]);
+        hv[k] = v * VN / d;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < RN_MAX_VEC; ++k)
+      if (hv[k] >= 0) {
+#pragma unroll
+        for (int i = 0; i < VN; ++i) ss[k] = fmaf(x[k][i], x[k][i], ss[k]);
+      }
+    float inv_mine[RN_MAX_VEC];
+#pragma unroll
+    for (int k = 0; k < RN_MAX_VEC; ++k) inv_mine[k] = 0.f;
+    for (int h = 0; h < H; ++h) {
+      float p = 0.f;
+#pragma unroll
+      for (int k = 0; k < RN_MAX_VEC; ++k) p += (hv[k] == h) ? ss[k] : 0.f;
+      p = warp_sum(p);
+      const float inv = 1.0f / fmaxf(sqrtf(p), 1e-12f);
+      if (mode == 0 && lane == 0) r_out[t * H + h] = inv;
+#pragma unroll
+      for (int k = 0; k < RN_MAX_VEC; ++k)
+        if (hv[k] == h) inv_mine[k] = inv;
+    }
+    if (mode == 1) {
+#pragma unroll
+      for (int k = 0; k < RN_MAX_VEC; ++k)
+        if (hv[k] >= 0) {
+#pragma unroll
+          for (int i = 0; i < VN; ++i) x[k][i] *= inv_mine[k];
+          store16(row + (lane + 32 * k) * VN, x[k]);
+        }
     }
   }
 }
 
 // ---------------------------------------------------------------------------
 // ShortConv2D (VGG-T3 key design 2): depthwise 3x3 zero-padded cross-correlation
-// per frame on the (N, h, w, C) patch grid.  threadIdx.x picks a 16-byte channel
-// vector (its 9*VN taps stay in registers), the y-dimension walks tokens.
+// per frame on the (N, h, w, C) patch grid.  CTA = (frame, 64-channel group);
+// it slides down the frame keeping rows y-1, y, y+1 of its channels in shared
+// memory (with zero columns at x = -1 and x = w), so every input element is
+// read from HBM once.  threadIdx.x = 16-byte channel vector within the group,
+// threadIdx.y = x position (strided by blockDim.y).
+
+constexpr int CONV_GROUP = 64;    // channels per CTA
+constexpr int CONV_MAX_W = 256;   // grid width limit of this kernel
 
 template <typename T>
-__global__ void k_shortconv(const T* __restrict__ V, int64_t ldv, T* __restrict__ out, int64_t ldo,
-                            const float* __restrict__ taps, int N, int gh, int gw, int C, int act) {
+__global__ void __launch_bounds__(256) k_shortconv(const T* __restrict__ V, int64_t ldv, T* __restrict__ out, int64_t ldo,
+                                                   const float* __restrict__ taps, int N, int gh, int gw, int C, int act) {
   constexpr int VN = Vec16<T>::N;
-  const int cv = blockIdx.x * blockDim.x + threadIdx.x;  // channel vector
-  if (cv * VN >= C) return;
-  const int c0 = cv * VN;
+  extern __shared__ float conv_sm[];   // [3][gw + 2][CONV_GROUP] fp32
+  const int n = blockIdx.x;
+  const int c0 = blockIdx.y * CONV_GROUP + threadIdx.x * VN;
+  const bool cvalid = c0 < C;
   float w[9][VN];
 #pragma unroll
   for (int i = 0; i < VN; ++i)
 #pragma unroll
-    for (int k = 0; k < 9; ++k) w[k][i] = taps[(c0 + i) * 9 + k];
-  const int64_t ntok = (int64_t)N * gh * gw;
-  for (int64_t t = (int64_t)blockIdx.y * blockDim.y + threadIdx.y; t < ntok; t += (int64_t)gridDim.y * blockDim.y) {
-    const int x = (int)(t % gw);
-    const int y = (int)((t / gw) % gh);
-    float acc[VN];
+    for (int k = 0; k < 9; ++k) w[k][i] = cvalid ? taps[(c0 + i) * 9 + k] : 0.f;
+  const int W2 = gw + 2;
+  auto slot = [&](int r, int x) { return conv_sm + ((size_t)(r % 3) * W2 + (x + 1)) * CONV_GROUP + threadIdx.x * VN; };
+  // zero the padding columns of all three row slots and prefill rows -1 (zeros) and 0
+  for (int r = 0; r < 3; ++r)
+    if (threadIdx.y == 0) {
 #pragma unroll
-    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-#pragma unroll
-    for (int dy = -1; dy <= 1; ++dy) {
-      if (y + dy < 0 || y + dy >= gh) continue;
-#pragma unroll
-      for (int dx = -1; dx <= 1; ++dx) {
-        if (x + dx < 0 || x + dx >= gw) continue;
-        float v[VN];
-        load16(V + (t + (int64_t)dy * gw + dx) * ldv + c0, v);
-        const int k = (dy + 1) * 3 + (dx + 1);
-#pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[k][i], v[i], acc[i]);
+      for (int i = 0; i < VN; ++i) {
+        slot(r, -1)[i] = 0.f;
+        slot(r, gw)[i] = 0.f;
       }
     }
-    if (act == 1) {
+  const int64_t frame0 = (int64_t)n * gh * gw;
+  auto load_row = [&](int y) {  // row y into slot y % 3 (zeros outside the frame)
+    for (int x = threadIdx.y; x < gw; x += blockDim.y) {
+      float v[VN];
+      if (y >= 0 && y < gh && cvalid) {
+        load16(V + (frame0 + (int64_t)y * gw + x) * ldv + c0, v);
+      } else {
 #pragma unroll
-      for (int i = 0; i < VN; ++i) acc[i] = acc[i] / (1.0f + expf(-acc[i]));
+        for (int i = 0; i < VN; ++i) v[i] = 0.f;
+      }
+      float* dst = slot(y + 3, x);
+#pragma unroll
+      for (int i = 0; i < VN; ++i) dst[i] = v[i];
     }
-    store16(out + t * ldo + c0, acc);
+  };
+  load_row(-1);
+  load_row(0);
+  for (int y = 0; y < gh; ++y) {
+    load_row(y + 1);
+    __syncthreads();
+    for (int x = threadIdx.y; x < gw; x += blockDim.y) {
+      float acc[VN];
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int dy = -1; dy <= 1; ++dy)
+#pragma unroll
+        for (int dx = -1; dx <= 1; ++dx) {
+          const float* src = slot(y + dy + 3, x + dx);
+          const int k = (dy + 1) * 3 + (dx + 1);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[k][i], src[i], acc[i]);
+        }
+      if (act == 1) {
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[i] = acc[i] / (1.0f + expf(-acc[i]));
+      }
+      if (cvalid) store16(out + (frame0 + (int64_t)y * gw + x) * ldo + c0, acc);
+    }
+    __syncthreads();
   }
 }
 
@@ -194,23 +282,40 @@ __device__ __forceinline__ void mat_shape(int b, int H, int d, int m, int& R, in
   if (b < 2 * H) { R = m; C = d; } else { R = d; C = m; }
 }
 
-__global__ void __launch_bounds__(256) k_frob_norms(const float* __restrict__ src, int64_t n_per, float* __restrict__ out) {
+constexpr int NORM_PARTS = 16;  // slices per matrix for the norm reductions
+
+// partial sums of squares: out[b * NORM_PARTS + p] over slice p of matrix b (n_per % 4 == 0)
+__global__ void __launch_bounds__(256) k_frob_partials(const float* __restrict__ src, int64_t n_per,
+                                                       float* __restrict__ out) {
   __shared__ float red[9];
-  const float* p = src + (int64_t)blockIdx.x * n_per;
+  const int b = blockIdx.x, p = blockIdx.y;
+  const int64_t n4 = n_per / 4, per = (n4 + NORM_PARTS - 1) / NORM_PARTS;
+  const int64_t i0 = p * per, i1 = min(n4, i0 + per);
+  const float4* x = reinterpret_cast<const float4*>(src + (int64_t)b * n_per);
   float s = 0.f;
-  for (int64_t i = threadIdx.x; i < n_per; i += 256) s = fmaf(p[i], p[i], s);
+  for (int64_t i = i0 + threadIdx.x; i < i1; i += 256) {
+    const float4 v = x[i];
+    s = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, s))));
+  }
   s = block_sum_256(s, red);
-  if (threadIdx.x == 0) out[blockIdx.x] = sqrtf(s);
+  if (threadIdx.x == 0) out[b * NORM_PARTS + p] = s;
 }
 
-__global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, const float* __restrict__ norms, int H,
+__device__ __forceinline__ float sum_parts(const float* parts) {
+  float s = 0.f;
+#pragma unroll
+  for (int p = 0; p < NORM_PARTS; ++p) s += parts[p];
+  return s;
+}
+
+__global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, const float* __restrict__ parts, int H,
                           int d, int m, float eps) {
   const int b = blockIdx.y;
   int R, C;
   mat_shape(b, H, d, m, R, C);
   const bool tall = R > C;
   const int64_t n = (int64_t)m * d;
-  const float sc = 1.0f / (norms[b] + eps);
+  const float sc = 1.0f / (sqrtf(sum_parts(parts + b * NORM_PARTS)) + eps);
   const float* g = G + (int64_t)b * n;
   float* x = X + (int64_t)b * n;
   const int c = tall ? R : C;  // columns of X
@@ -221,60 +326,110 @@ __global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, co
   }
 }
 
-// Batched C = alpha * A * op(B) + beta * Cin, fp32, 64x64 tiles, 256 threads.
+// Delta in W's orientation: D_b = X_b for wide matrices, X_b^T for tall ones (32x32 smem tiles).
+// grid (ceil(C/32), ceil(R/32), 3H) over W's shape (R, C); block (32, 8).
+__global__ void k_ns_finish(const float* __restrict__ X, float* __restrict__ D, int H, int d, int m) {
+  __shared__ float tile[32][33];
+  const int b = blockIdx.z;
+  int R, C;
+  mat_shape(b, H, d, m, R, C);
+  const int64_t n = (int64_t)m * d;
+  const float* x = X + (int64_t)b * n;
+  float* o = D + (int64_t)b * n;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  if (r0 >= R || c0 >= C) return;
+  if (R <= C) {
+    for (int yy = threadIdx.y; yy < 32; yy += 8) {
+      const int r = r0 + yy, c = c0 + threadIdx.x;
+      if (r < R && c < C) o[(int64_t)r * C + c] = x[(int64_t)r * C + c];
+    }
+    return;
+  }
+  // tall: X is (C, R); D[r][c] = X[c][r]
+  for (int yy = threadIdx.y; yy < 32; yy += 8) {
+    const int xc = c0 + yy, xr = r0 + threadIdx.x;  // X row xc, column xr
+    tile[yy][threadIdx.x] = (xc < C && xr < R) ? x[(int64_t)xc * R + xr] : 0.f;
+  }
+  __syncthreads();
+  for (int yy = threadIdx.y; yy < 32; yy += 8) {
+    const int r = r0 + yy, c = c0 + threadIdx.x;
+    if (r < R && c < C) o[(int64_t)r * C + c] = tile[threadIdx.x][yy];
+  }
+}
+
+// Batched C = alpha * A * op(B) + beta * Cin, fp32, 64x64 tiles, 256 threads, 4x4 per thread.
 // A: [M][K] (lda), op(B) = B [K][N] (ldb) or, with TRANS_B, B^T with B [N][K].
+// Global loads of the next 16-deep K slice are issued before the current slice's FMAs.
 template <bool TRANS_B>
 __global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const float* __restrict__ A, int lda, int64_t sA,
                                                   const float* __restrict__ B, int ldb, int64_t sB, float* __restrict__ C,
                                                   int ldc, int64_t sC, const float* __restrict__ Cin, float alpha,
                                                   float beta) {
-  __shared__ float As[16][64 + 4];
-  __shared__ float Bs[16][64 + 4];
+  __shared__ __align__(16) float As[2][16][64];
+  __shared__ __align__(16) float Bs[2][16][64];
   const int b = blockIdx.z;
   A += b * sA;
   B += b * sB;
   C += b * sC;
   if (Cin) Cin += b * sC;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
-      const int kk = i & 15, mm = i >> 4;
-      const int gm = m0 + mm, gk = k0 + kk;
-      As[kk][mm] = (gm < M && gk < K) ? A[(int64_t)gm * lda + gk] : 0.f;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // loader mapping: 4 elements per thread per operand per slice
+  float ra[4], rb[4];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = tid + 256 * q;
+      {  // A slice [64 m][16 k]: i -> (mm = i / 16, kk = i % 16)
+        const int kk = i & 15, mm = i >> 4, gm = m0 + mm, gk = k0 + kk;
+        ra[q] = (gm < M && gk < K) ? A[(int64_t)gm * lda + gk] : 0.f;
+      }
       if (TRANS_B) {
-        const int gn = n0 + mm;
-        Bs[kk][mm] = (gn < N && gk < K) ? B[(int64_t)gn * ldb + gk] : 0.f;
+        const int kk = i & 15, nn = i >> 4, gn = n0 + nn, gk = k0 + kk;
+        rb[q] = (gn < N && gk < K) ? B[(int64_t)gn * ldb + gk] : 0.f;
+      } else {
+        const int nn = i & 63, kk = i >> 6, gn = n0 + nn, gk = k0 + kk;
+        rb[q] = (gn < N && gk < K) ? B[(int64_t)gk * ldb + gn] : 0.f;
       }
     }
-    if (!TRANS_B) {
-      for (int i = threadIdx.x; i < 16 * 64; i += 256) {
-        const int nn = i & 63, kk = i >> 6;
-        const int gn = n0 + nn, gk = k0 + kk;
-        Bs[kk][nn] = (gn < N && gk < K) ? B[(int64_t)gk * ldb + gn] : 0.f;
-      }
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = tid + 256 * q;
+      As[buf][i & 15][i >> 4] = ra[q];
+      if (TRANS_B) Bs[buf][i & 15][i >> 4] = rb[q];
+      else Bs[buf][i >> 6][i & 63] = rb[q];
     }
-    __syncthreads();
+  };
+  float acc[4][4] = {};
+  load(0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    const bool more = k0 + 16 < K;
+    if (more) load(k0 + 16);
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
-      float a[4], bb[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx + 16 * j];
+      const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float a4[4] = {av.x, av.y, av.z, av.w};
+      const float b4[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
     }
+    if (more) stash(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int gm = m0 + ty + 16 * i, gn = n0 + tx + 16 * j;
+      const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
       if (gm < M && gn < N) {
         float v = alpha * acc[i][j];
         if (Cin) v = fmaf(beta, Cin[(int64_t)gm * ldc + gn], v);
@@ -284,58 +439,62 @@ __global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const flo
 }
 
 // ---------------------------------------------------------------------------
-// Muon weight step (ZipMap key design 3): W <- ||W|| (W - lr D) / ||W - lr D||.
-// D_b is read from X_b (wide orientation, transposed back for tall matrices),
-// or from G_b directly when Newton-Schulz is disabled (iters = 0).
-
-__device__ __forceinline__ float delta_at(const float* __restrict__ D, int b, int64_t i, int H, int d, int m,
-                                          bool from_x) {
-  const int64_t n = (int64_t)m * d;
-  if (!from_x) return D[(int64_t)b * n + i];
-  int R, C;
-  mat_shape(b, H, d, m, R, C);
-  if (R <= C) return D[(int64_t)b * n + i];
-  const int64_t ri = i / C, cj = i % C;  // W index (ri, cj) -> X (cj, ri), X has R columns
-  return D[(int64_t)b * n + cj * R + ri];
-}
+// Muon weight step (ZipMap key design 3): W <- ||W|| (W - lr D) / ||W - lr D||,
+// D in W's orientation (k_ns_finish), or G itself when Newton-Schulz is off.
 
 __device__ __forceinline__ float* mat_ptr(float* W1, float* W3, float* W2, int b, int H, int64_t n) {
   return b < H ? W1 + (int64_t)b * n : (b < 2 * H ? W3 + (int64_t)(b - H) * n : W2 + (int64_t)(b - 2 * H) * n);
 }
 
-__global__ void __launch_bounds__(256) k_step_norms(float* W1, float* W3, float* W2, const float* __restrict__ D, int H,
-                                                    int d, int m, float lr, int from_x, float* __restrict__ out) {
+// partials out[(b * NORM_PARTS + p) * 2 + {0,1}] of ||W_b||^2 and ||W_b - lr D_b||^2
+__global__ void __launch_bounds__(256) k_step_partials(float* W1, float* W3, float* W2, const float* __restrict__ D,
+                                                       int H, int d, int m, float lr, float* __restrict__ out) {
   __shared__ float red[9];
-  const int b = blockIdx.x;
-  const int64_t n = (int64_t)m * d;
-  const float* w = mat_ptr(W1, W3, W2, b, H, n);
+  const int b = blockIdx.x, p = blockIdx.y;
+  const int64_t n = (int64_t)m * d, n4 = n / 4, per = (n4 + NORM_PARTS - 1) / NORM_PARTS;
+  const int64_t i0 = p * per, i1 = min(n4, i0 + per);
+  const float4* w = reinterpret_cast<const float4*>(mat_ptr(W1, W3, W2, b, H, n));
+  const float4* dl = reinterpret_cast<const float4*>(D + (int64_t)b * n);
   float s0 = 0.f, s1 = 0.f;
-  for (int64_t i = threadIdx.x; i < n; i += 256) {
-    const float wi = w[i];
-    const float u = wi - lr * delta_at(D, b, i, H, d, m, from_x != 0);
-    s0 = fmaf(wi, wi, s0);
-    s1 = fmaf(u, u, s1);
+  for (int64_t i = i0 + threadIdx.x; i < i1; i += 256) {
+    const float4 a = w[i], q = dl[i];
+    const float u0 = a.x - lr * q.x, u1 = a.y - lr * q.y, u2 = a.z - lr * q.z, u3 = a.w - lr * q.w;
+    s0 = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, s0))));
+    s1 = fmaf(u0, u0, fmaf(u1, u1, fmaf(u2, u2, fmaf(u3, u3, s1))));
   }
   s0 = block_sum_256(s0, red);
   s1 = block_sum_256(s1, red);
   if (threadIdx.x == 0) {
-    out[2 * b] = sqrtf(s0);
-    out[2 * b + 1] = sqrtf(s1);
+    out[(b * NORM_PARTS + p) * 2] = s0;
+    out[(b * NORM_PARTS + p) * 2 + 1] = s1;
   }
 }
 
 __global__ void k_step_apply(float* W1, float* W3, float* W2, const float* __restrict__ D, int H, int d, int m, float lr,
-                             int from_x, int renorm, const float* __restrict__ norms) {
+                             int renorm, const float* __restrict__ parts) {
   const int b = blockIdx.y;
-  const int64_t n = (int64_t)m * d;
-  float* w = mat_ptr(W1, W3, W2, b, H, n);
+  const int64_t n = (int64_t)m * d, n4 = n / 4;
+  float4* w = reinterpret_cast<float4*>(mat_ptr(W1, W3, W2, b, H, n));
+  const float4* dl = reinterpret_cast<const float4*>(D + (int64_t)b * n);
   float sc = 1.f;
   if (renorm) {
-    const float nu = norms[2 * b + 1];
-    sc = nu > 0.f ? norms[2 * b] / nu : 1.f;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int p = 0; p < NORM_PARTS; ++p) {
+      s0 += parts[(b * NORM_PARTS + p) * 2];
+      s1 += parts[(b * NORM_PARTS + p) * 2 + 1];
+    }
+    sc = s1 > 0.f ? sqrtf(s0) / sqrtf(s1) : 1.f;
   }
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    w[i] = sc * (w[i] - lr * delta_at(D, b, i, H, d, m, from_x != 0));
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    float4 a = w[i];
+    const float4 q = dl[i];
+    a.x = sc * (a.x - lr * q.x);
+    a.y = sc * (a.y - lr * q.y);
+    a.z = sc * (a.z - lr * q.z);
+    a.w = sc * (a.w - lr * q.w);
+    w[i] = a;
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -36,11 +36,18 @@ constexpr int TC_BLK = 128 * 128;   // one [128 rows x 64 bf16] swizzled block
 template <int D>
 struct UpdLayout {
   static constexpr int KB = D / 64;               // 64-wide d blocks
+  static constexpr int NFB = 2 * KB;              // forward blocks per tile: K blocks, then V blocks
+  static constexpr int NF = 3;                    // forward ring stages ([128 tok x 64 d] each)
+  static constexpr int BCH = 32;                  // tokens per backward stage
+  static constexpr int NBC = TC_TILE / BCH;       // backward stages per tile
+  static constexpr int NB = 2;                    // backward ring stages
   static constexpr int W_BLK = 3 * 64 * 128;      // per d block: W1s, W3s, W2s^T rows (64 each)
+  static constexpr int BCHUNK = BCH * 128;        // [32 tok x 64 d] swizzled
+  static constexpr int BSTAGE = 2 * KB * BCHUNK;  // K chunks (KB) then V chunks (KB)
   static constexpr int W_OFF = 0;
-  static constexpr int K_OFF = W_OFF + KB * W_BLK;
-  static constexpr int V_OFF = K_OFF + KB * TC_BLK;
-  static constexpr int DH_OFF = V_OFF + KB * TC_BLK;  // [dH1 block | dH3 block]
+  static constexpr int F_OFF = W_OFF + KB * W_BLK;
+  static constexpr int B_OFF = F_OFF + NF * TC_BLK;
+  static constexpr int DH_OFF = B_OFF + NB * BSTAGE;  // [dH1 block | dH3 block]
   static constexpr int U_OFF = DH_OFF + 2 * TC_BLK;
   static constexpr int BAR_OFF = U_OFF + TC_BLK;
   static constexpr int BYTES = BAR_OFF + 256;
@@ -49,11 +56,29 @@ struct UpdLayout {
   static constexpr int G2_COL = 192 + D;
   static constexpr int N_G2 = (D == 192) ? 2 : 1;
   static_assert(G2_COL + 64 * N_G2 <= 512, "TMEM budget");
+  static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
+constexpr int UPD_THREADS = 352;  // warp 0: forward TMA, 1: MMA, 2..9: epilogue, 10: backward TMA
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Streaming gradient kernel.  Per 128-token tile i the tensor pipe runs the
+// forward F_i (H1|H3 and Z from K, V d-blocks streamed through the forward ring)
+// and the backward G_i (gradient GEMMs from K, V token chunks streamed a second
+// time through the backward ring, with dH/U~ from shared memory).  The epilogue
+// drains F_i from TMEM into registers first and releases it, so F_(i+1) runs
+// while the epilogue computes; G_i is interleaved with F_(i+1) once the
+// epilogue has written dH_i.  K and V are read twice from L2 (once per ring),
+// which buys the latency hiding that a single resident tile cannot.
 template <int D>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(UPD_THREADS, 1)
     k_update_grad_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                      const __grid_constant__ CUtensorMap tmW, const float* __restrict__ eta,
                      const float* __restrict__ rk, float* __restrict__ partial, int64_t T, int H, int m,
                      int tiles_total, int S, unsigned int* status, unsigned long long timeout_ns) {
@@ -68,22 +93,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* wfull = bars + 0;
-  uint64_t* kfull = bars + 1;
-  uint64_t* vfull = bars + 2;
-  uint64_t* kfree = bars + 3;
-  uint64_t* vfree = bars + 4;
-  uint64_t* fdone = bars + 5;
-  uint64_t* edone = bars + 6;
-  uint64_t* gdone = bars + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint64_t* ffull = bars + 1;             // [NF]
+  uint64_t* fempty = ffull + L::NF;       // [NF]
+  uint64_t* bfull = fempty + L::NF;       // [NB]
+  uint64_t* bempty = bfull + L::NB;       // [NB]
+  uint64_t* fdone = bempty + L::NB;       // forward of a tile complete (TMEM F valid)
+  uint64_t* ffree = fdone + 1;            // epilogue drained F (256 arrivals)
+  uint64_t* edone = ffree + 1;            // epilogue wrote dH, U~ (256 arrivals)
+  uint64_t* gdone = edone + 1;            // backward of a tile complete (dH buffer reusable)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gdone + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(wfull, 1);
-    mbar_init(kfull, 1);
-    mbar_init(vfull, 1);
-    mbar_init(kfree, 1);
-    mbar_init(vfree, 1);
+    for (int i = 0; i < L::NF; ++i) {
+      mbar_init(ffull + i, 1);
+      mbar_init(fempty + i, 1);
+    }
+    for (int i = 0; i < L::NB; ++i) {
+      mbar_init(bfull + i, 1);
+      mbar_init(bempty + i, 1);
+    }
     mbar_init(fdone, 1);
+    mbar_init(ffree, 256);
     mbar_init(edone, 256);
     mbar_init(gdone, 1);
     fence_mbar_init();
@@ -100,7 +131,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- forward ring producer: W once, then per tile K blocks then V blocks
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmW);
@@ -111,71 +142,123 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tma_load_2d(dst + 8192, &tmW, wfull, kb * 64, H * m + h * m + slice * TC_MS);
         tma_load_2d(dst + 16384, &tmW, wfull, kb * 64, 2 * H * m + h * m + slice * TC_MS);
       }
-      for (int i = 0; i < ntiles; ++i) {
+      int fc = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < ntiles; ++i) {
         const int t0 = (t_begin + i) * TC_TILE;
-        if (i > 0 && !mbar_wait(kfree, (i - 1) & 1, g)) break;
-        mbar_expect_tx(kfull, L::KB * TC_BLK);
-        for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_2d(smem + L::K_OFF + kb * TC_BLK, &tmK, kfull, h * D + kb * 64, t0);
-        if (i > 0 && !mbar_wait(vfree, (i - 1) & 1, g)) break;
-        mbar_expect_tx(vfull, L::KB * TC_BLK);
-        for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_2d(smem + L::V_OFF + kb * TC_BLK, &tmV, vfull, h * D + kb * 64, t0);
+        for (int b = 0; b < L::NFB; ++b, ++fc) {
+          const int st = fc % L::NF, use = fc / L::NF;
+          if (use > 0 && !mbar_wait(fempty + st, (use - 1) & 1, g)) { ok = false; break; }
+          mbar_expect_tx(ffull + st, TC_BLK);
+          const bool isk = b < L::KB;
+          tma_load_2d(smem + L::F_OFF + st * TC_BLK, isk ? &tmK : &tmV, ffull + st, h * D + (isk ? b : b - L::KB) * 64,
+                      t0);
+        }
+      }
+    }
+  } else if (warp == 10) {
+    if (lane == 0) {
+      // ---------------- backward ring producer: per tile, 32-token chunks of K and V (all d)
+      tma_prefetch_desc(&tmKb);
+      tma_prefetch_desc(&tmVb);
+      int bc = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int t0 = (t_begin + i) * TC_TILE;
+        for (int c = 0; c < L::NBC; ++c, ++bc) {
+          const int st = bc % L::NB, use = bc / L::NB;
+          if (use > 0 && !mbar_wait(bempty + st, (use - 1) & 1, g)) { ok = false; break; }
+          mbar_expect_tx(bfull + st, L::BSTAGE);
+          uint8_t* dst = smem + L::B_OFF + st * L::BSTAGE;
+          for (int kb = 0; kb < L::KB; ++kb) {
+            tma_load_2d(dst + kb * L::BCHUNK, &tmKb, bfull + st, h * D + kb * 64, t0 + c * L::BCH);
+            tma_load_2d(dst + (L::KB + kb) * L::BCHUNK, &tmVb, bfull + st, h * D + kb * 64, t0 + c * L::BCH);
+          }
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      const uint32_t sW = smem_u32(smem + L::W_OFF), sK = smem_u32(smem + L::K_OFF);
-      const uint32_t sV = smem_u32(smem + L::V_OFF), sDH = smem_u32(smem + L::DH_OFF);
+      const uint32_t sW = smem_u32(smem + L::W_OFF), sF = smem_u32(smem + L::F_OFF);
+      const uint32_t sB = smem_u32(smem + L::B_OFF), sDH = smem_u32(smem + L::DH_OFF);
       const uint32_t sU = smem_u32(smem + L::U_OFF);
       constexpr uint32_t ID_F13 = idesc_bf16(128, 128, false, false);
       constexpr uint32_t ID_Z = idesc_bf16(128, 64, false, false);
       constexpr uint32_t ID_G13 = idesc_bf16(128, D, true, true);
       constexpr uint32_t ID_G2 = idesc_bf16(128, 64, true, true);
-      bool ok = mbar_wait(wfull, 0, g);
-      for (int i = 0; ok && i < ntiles; ++i) {
-        const uint32_t ph = i & 1;
-        if (!mbar_wait(kfull, ph, g)) break;
+      int fc = 0, bc = 0;
+      // one forward block b of the current forward tile
+      auto f_block = [&](int b) -> bool {
+        const int st = fc % L::NF, use = fc / L::NF;
+        if (!mbar_wait(ffull + st, use & 1, g)) return false;
         tc_fence_after();
-        // [H1 | H3] = K [W1s; W3s]^T : M=128 tokens, N=128, K=D (A, B K-major)
+        const uint32_t a0 = sF + st * TC_BLK;
+        if (b < L::KB) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const int kb = ks >> 2, kw = ks & 3;
-          umma_bf16_ss(tmem + 0, sdesc_sw128(sK + kb * TC_BLK + kw * 32, 16, 1024),
-                       sdesc_sw128(sW + kb * L::W_BLK + kw * 32, 16, 1024), ID_F13, ks > 0);
+          for (int kw = 0; kw < 4; ++kw)
+            umma_bf16_ss(tmem + 0, sdesc_sw128(a0 + kw * 32, 16, 1024),
+                         sdesc_sw128(sW + b * L::W_BLK + kw * 32, 16, 1024), ID_F13, (b > 0 || kw > 0));
+        } else {
+          const int vb = b - L::KB;
+#pragma unroll
+          for (int kw = 0; kw < 4; ++kw)
+            umma_bf16_ss(tmem + 128, sdesc_sw128(a0 + kw * 32, 16, 1024),
+                         sdesc_sw128(sW + vb * L::W_BLK + 16384 + kw * 32, 16, 1024), ID_Z, (vb > 0 || kw > 0));
         }
-        if (!mbar_wait(vfull, ph, g)) break;
+        umma_commit(fempty + st);
+        ++fc;
+        return true;
+      };
+      // one backward chunk c of tile i (dH/U~ of tile i must be in shared memory)
+      auto g_chunk = [&](int i, int c) -> bool {
+        const int st = bc % L::NB, use = bc / L::NB;
+        if (!mbar_wait(bfull + st, use & 1, g)) return false;
         tc_fence_after();
-        // Z = V W2s : B = W2s^T rows (K-major)
+        const uint32_t b0 = sB + st * L::BSTAGE;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const int kb = ks >> 2, kw = ks & 3;
-          umma_bf16_ss(tmem + 128, sdesc_sw128(sV + kb * TC_BLK + kw * 32, 16, 1024),
-                       sdesc_sw128(sW + kb * L::W_BLK + 16384 + kw * 32, 16, 1024), ID_Z, ks > 0);
-        }
-        umma_commit(fdone);
-        if (!mbar_wait(edone, ph, g)) break;
-        tc_fence_after();
-        // [g1s; g3s] += [dH1 | dH3]^T K : M=128 (stacked m rows), N=D, K=128 tokens (A, B MN-major)
-#pragma unroll
-        for (int ks = 0; ks < TC_TILE / 16; ++ks) {
+        for (int j = 0; j < L::BCH / 16; ++j) {
+          const int ks = c * (L::BCH / 16) + j;
+          const uint32_t acc = (i > 0 || ks > 0);
           umma_bf16_ss(tmem + L::G13_COL, sdesc_sw128(sDH + ks * 2048, TC_BLK, 1024),
-                       sdesc_sw128(sK + ks * 2048, TC_BLK, 1024), ID_G13, (i > 0 || ks > 0));
+                       sdesc_sw128(b0 + j * 2048, L::BCHUNK, 1024), ID_G13, acc);
+#pragma unroll
+          for (int rb = 0; rb < L::N_G2; ++rb)
+            umma_bf16_ss(tmem + L::G2_COL + rb * 64,
+                         sdesc_sw128(b0 + (L::KB + rb) * L::BCHUNK + j * 2048, L::BCHUNK, 1024),
+                         sdesc_sw128(sU + ks * 2048, TC_BLK, 1024), ID_G2, acc);
         }
-        umma_commit(kfree);
-        // g2[rows, s] += V[:, rows]^T U~ : M=128 d rows, N=64, K=128 tokens (A, B MN-major)
-#pragma unroll
-        for (int rb = 0; rb < L::N_G2; ++rb) {
-#pragma unroll
-          for (int ks = 0; ks < TC_TILE / 16; ++ks) {
-            umma_bf16_ss(tmem + L::G2_COL + rb * 64, sdesc_sw128(sV + rb * TC_BLK + ks * 2048, TC_BLK, 1024),
-                         sdesc_sw128(sU + ks * 2048, TC_BLK, 1024), ID_G2, (i > 0 || ks > 0));
+        umma_commit(bempty + st);
+        ++bc;
+        return true;
+      };
+      bool ok = mbar_wait(wfull, 0, g);
+      if (ok && ntiles > 0) {
+        for (int b = 0; ok && b < L::NFB; ++b) ok = f_block(b);
+        if (ok) umma_commit(fdone);
+      }
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const bool has_next = i + 1 < ntiles;
+        // F_(i+1) may overwrite TMEM F once the epilogue has drained F_i
+        if (has_next && !mbar_wait(ffree, i & 1, g)) break;
+        // the first forward blocks cover the epilogue's compute, then F and G alternate
+        int fb = 0, gcn = 0;
+        const int lead = has_next ? (L::NFB < 3 ? L::NFB : 3) : 0;
+        for (; ok && fb < lead; ++fb) ok = f_block(fb);
+        if (!ok) break;
+        if (has_next && fb == L::NFB) umma_commit(fdone);
+        if (!mbar_wait(edone, i & 1, g)) break;
+        tc_fence_after();
+        while (ok && (gcn < L::NBC || (has_next && fb < L::NFB))) {
+          if (gcn < L::NBC) ok = g_chunk(i, gcn++);
+          if (ok && has_next && fb < L::NFB) {
+            ok = f_block(fb++);
+            if (ok && fb == L::NFB) umma_commit(fdone);
           }
         }
-        umma_commit(vfree);
+        if (!ok) break;
+        umma_commit(gdone);
       }
-      umma_commit(gdone);
     }
   } else {
     // ---------------- epilogue warps 2..9
@@ -200,26 +283,36 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tmem_ld_wait(a1);
       tmem_ld_wait(a3);
       tmem_ld_wait(az);
+      tc_fence_before();
+      mbar_arrive(ffree);  // F may now be overwritten by the next tile's forward
+      const float2 r2 = make_float2(r, r);
+      const float2 er2 = make_float2(-e * r, -e * r);   // -eta * r
+      const float2 ne2 = make_float2(-e, -e);
+      const float2 half2 = make_float2(0.5f, 0.5f);
+      const float2 one2 = make_float2(1.f, 1.f);
       uint32_t p1[16], p3[16], pu[16];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
-        float o1[2], o3[2], ou[2];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const float h1 = __uint_as_float(a1[j + k]) * r;
-          const float h3 = __uint_as_float(a3[j + k]) * r;
-          const float z = __uint_as_float(az[j + k]);
-          const float s = 1.0f / (1.0f + __expf(-h1));
-          const float a = h1 * s;
-          const float du = -e * z;
-          o1[k] = du * h3 * s * (1.0f + h1 * (1.0f - s)) * r;  // dL/dh1 chained to the raw key
-          o3[k] = du * a * r;                                   // dL/dh3 chained to the raw key
-          ou[k] = -e * a * h3;                                  // -eta u
-        }
-        p1[j >> 1] = pack_bf16x2(o1[0], o1[1]);
-        p3[j >> 1] = pack_bf16x2(o3[0], o3[1]);
-        pu[j >> 1] = pack_bf16x2(ou[0], ou[1]);
+        const float2 h1 = __fmul2_rn(make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1])), r2);
+        const float2 h3 = __fmul2_rn(make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1])), r2);
+        const float2 z = make_float2(__uint_as_float(az[j]), __uint_as_float(az[j + 1]));
+        const float2 hh = __fmul2_rn(h1, half2);
+        const float2 th = make_float2(tanh_approx(hh.x), tanh_approx(hh.y));
+        const float2 s = __ffma2_rn(th, half2, half2);           // sigmoid(h1)
+        const float2 a = __fmul2_rn(h1, s);                      // SiLU(h1)
+        const float2 u = __fmul2_rn(a, h3);
+        const float2 dz = __fmul2_rn(er2, z);                    // dL/du chained to the raw key
+        const float2 oms = __fadd2_rn(one2, make_float2(-s.x, -s.y));
+        const float2 qd = __ffma2_rn(a, oms, s);                 // SiLU'(h1) = s + a (1 - s)
+        const float2 d1 = __fmul2_rn(__fmul2_rn(dz, h3), qd);    // dL/dh1 (raw key)
+        const float2 d3 = __fmul2_rn(dz, a);                     // dL/dh3 (raw key)
+        const float2 ut = __fmul2_rn(ne2, u);                    // -eta u
+        p1[j >> 1] = pack_bf16x2(d1.x, d1.y);
+        p3[j >> 1] = pack_bf16x2(d3.x, d3.y);
+        pu[j >> 1] = pack_bf16x2(ut.x, ut.y);
       }
+      // dH / U~ buffer is free once the previous tile's backward has completed
+      if (i > 0 && !__all_sync(0xffffffffu, mbar_wait(gdone, (i - 1) & 1, g))) { ok = false; break; }
       uint8_t* sdh = smem + L::DH_OFF;
       uint8_t* su = smem + L::U_OFF;
 #pragma unroll
@@ -231,10 +324,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         *reinterpret_cast<uint4*>(su + off) = make_uint4(pu[4 * c], pu[4 * c + 1], pu[4 * c + 2], pu[4 * c + 3]);
       }
       fence_async_smem();
-      tc_fence_before();
       mbar_arrive(edone);
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(gdone, 0, g));
+    if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(gdone, (ntiles - 1) & 1, g));
     if (ok && ntiles == 0) {
       // empty token range: the gradient partial is zero
       const int64_t n = (int64_t)m * D;

@@ -80,8 +80,8 @@ struct Ws {
   float* X2;           // [3H][m*d]
   float* A;            // [3H][r*r]
   float* B;            // [3H][r*r]
-  float* norms;        // [3H]
-  float* stepn;        // [2*3H]
+  float* norms;        // [3H][NORM_PARTS] partial sums of squares of G
+  float* stepn;        // [3H][NORM_PARTS][2] partials of ||W||^2, ||W - lr D||^2
   float* rk;           // [T][H]
   float* rq;           // [T][H]
   size_t total;
@@ -125,8 +125,8 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_X2 = take(3 * n * 4);
   const size_t o_A = take(3 * H * r * r * 4);
   const size_t o_B = take(3 * H * r * r * 4);
-  const size_t o_norms = take(3 * H * 4);
-  const size_t o_stepn = take(6 * H * 4);
+  const size_t o_norms = take(3 * H * NORM_PARTS * 4);
+  const size_t o_stepn = take(3 * H * NORM_PARTS * 2 * 4);
   const size_t o_rk = take((size_t)std::max<int64_t>(T, 1) * H * 4);
   const size_t o_rq = take((size_t)std::max<int64_t>(T, 1) * H * 4);
   w.total = off;
@@ -304,23 +304,25 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
     const int tiles = (int)((T + TC_TILE - 1) / TC_TILE);
     const int slices = d.m / TC_MS;
     S = std::max(1, std::min({sm_count() / std::max(1, slices * d.heads), w.s_max, tiles}));
-    CUtensorMap tK, tV, tW;
+    CUtensorMap tK, tV, tKb, tVb, tW;
     const uint64_t hd = (uint64_t)d.heads * d.d;
     if (!tmap_bf16(&tK, K, hd, (uint64_t)T, (uint64_t)ldk * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
     if (!tmap_bf16(&tV, V, hd, (uint64_t)T, (uint64_t)ldv * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tKb, K, hd, (uint64_t)T, (uint64_t)ldk * 2, 64, UpdLayout<192>::BCH)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tVb, V, hd, (uint64_t)T, (uint64_t)ldv * 2, 64, UpdLayout<192>::BCH)) return TTT_ERR_CUDA;
     if (!tmap_bf16(&tW, w.wsh, (uint64_t)d.d, 3ull * d.heads * d.m, (uint64_t)d.d * 2, 64, 64)) return TTT_ERR_CUDA;
     dim3 grid(slices, d.heads, S);
     ProfScope ps(TTT_PROF_GRAD, s);
     if (d.d == 192) {
       auto k = k_update_grad_tc<192>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<192>::ALLOC));
-      k<<<grid, TC_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tW, eta, rk, w.partial, T, d.heads, d.m, tiles, S,
-                                                         w.status, wait_timeout_ns());
+      k<<<grid, UPD_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, rk, w.partial, T, d.heads, d.m,
+                                                          tiles, S, w.status, wait_timeout_ns());
     } else {
       auto k = k_update_grad_tc<128>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<128>::ALLOC));
-      k<<<grid, TC_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tW, eta, rk, w.partial, T, d.heads, d.m, tiles, S,
-                                                         w.status, wait_timeout_ns());
+      k<<<grid, UPD_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, rk, w.partial, T, d.heads, d.m,
+                                                          tiles, S, w.status, wait_timeout_ns());
     }
     TTT_LAUNCHED();
   } else {
@@ -349,10 +351,9 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
   const int nb = 3 * H;
   const int r = std::min(mm, dd), c = std::max(mm, dd);
   const float* D = G;
-  int from_x = 0;
   ProfScope ps(TTT_PROF_NS, s);
   if (ns.iters > 0) {
-    k_frob_norms<<<nb, 256, 0, s>>>(G, n, w.norms);
+    k_frob_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(G, n, w.norms);
     TTT_LAUNCHED();
     k_ns_init<<<dim3(grid1d(n, 256) / nb + 1, nb), 256, 0, s>>>(G, w.X, w.norms, H, dd, mm, ns.eps);
     TTT_LAUNCHED();
@@ -371,13 +372,15 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
       TTT_LAUNCHED();
       std::swap(X, X2);
     }
-    D = X;
-    from_x = 1;
+    // Delta back in W's orientation, into the buffer X does not occupy
+    k_ns_finish<<<dim3((c + 31) / 32, (c + 31) / 32, nb), dim3(32, 8), 0, s>>>(X, X2, H, dd, mm);
+    TTT_LAUNCHED();
+    D = X2;
   }
-  k_step_norms<<<nb, 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, from_x, w.stepn);
+  k_step_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, w.stepn);
   TTT_LAUNCHED();
-  k_step_apply<<<dim3(grid1d(n, 256) / nb + 1, nb), 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, from_x,
-                                                                 ns.renorm, w.stepn);
+  k_step_apply<<<dim3(grid1d(n / 4, 256) / nb + 1, nb), 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, ns.renorm,
+                                                                    w.stepn);
   TTT_LAUNCHED();
   return TTT_OK;
 }
@@ -502,19 +505,22 @@ int ttt_shortconv2d(const void* V, int64_t ld_v, void* Vout, int64_t ld_out, con
   if (!V || !Vout || !taps || V == Vout) return TTT_ERR_INVALID;
   if (!aligned16(V) || !aligned16(Vout) || (ld_v * (int64_t)esize(dtype)) % 16 || (ld_out * (int64_t)esize(dtype)) % 16)
     return TTT_ERR_ALIGN;
+  if (w > CONV_MAX_W) return TTT_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
-  const int64_t ntok = (int64_t)N * h * w;
   const int vn = dtype == TTT_BF16 ? 8 : 4;
-  const int nvec = C / vn;
-  dim3 block(std::min(nvec, 128), std::max(1, 256 / std::min(nvec, 128)));
-  dim3 grid((nvec + block.x - 1) / block.x,
-            (unsigned)std::max<int64_t>(1, std::min<int64_t>((ntok + block.y - 1) / block.y, 65535)));
+  const int gv = CONV_GROUP / vn;
+  const dim3 block(gv, 256 / gv);
+  const dim3 grid(N, (C + CONV_GROUP - 1) / CONV_GROUP);
+  const size_t smem = (size_t)3 * (w + 2) * CONV_GROUP * sizeof(float);
   ProfScope ps(TTT_PROF_CONV, s);
-  if (dtype == TTT_BF16)
-    k_shortconv<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)V, ld_v, (__nv_bfloat16*)Vout, ld_out,
-                                                      taps, N, h, w, C, act);
-  else
-    k_shortconv<float><<<grid, block, 0, s>>>((const float*)V, ld_v, (float*)Vout, ld_out, taps, N, h, w, C, act);
+  if (dtype == TTT_BF16) {
+    TTT_CHECK(cudaFuncSetAttribute(k_shortconv<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_shortconv<__nv_bfloat16><<<grid, block, smem, s>>>((const __nv_bfloat16*)V, ld_v, (__nv_bfloat16*)Vout, ld_out,
+                                                         taps, N, h, w, C, act);
+  } else {
+    TTT_CHECK(cudaFuncSetAttribute(k_shortconv<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    k_shortconv<float><<<grid, block, smem, s>>>((const float*)V, ld_v, (float*)Vout, ld_out, taps, N, h, w, C, act);
+  }
   TTT_LAUNCHED();
   return TTT_OK;
 }
