@@ -390,18 +390,28 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
 template <int D>
 struct ApLayout {
   static constexpr int KB = D / 64;
-  static constexpr int Q_OFF = 0;
-  static constexpr int W13_BYTES = KB * TC_BLK;          // [W1c; W3c]: 128 rows per d block
-  static constexpr int W2_BYTES = D * 128;               // W2c: D rows x 64 m
-  static constexpr int STAGE = W13_BYTES + W2_BYTES;
+  static constexpr int Q_OFF = 0;                        // this CTA's 128 query tokens, all d
+  static constexpr int W13_HALF = KB * 64 * 128;         // this CTA's 64 rows of [W1c; W3c] (W1c or W3c)
+  static constexpr int W2_HALF = (D / 2) * 128;          // this CTA's D/2 rows of W2c (64 m each)
+  static constexpr int STAGE = W13_HALF + W2_HALF;
+  static constexpr int NS = 3;                           // weight ring stages
   static constexpr int W_OFF = Q_OFF + KB * TC_BLK;
-  static constexpr int P_OFF = W_OFF + 2 * STAGE;
+  static constexpr int P_OFF = W_OFF + NS * STAGE;
   static constexpr int BAR_OFF = P_OFF + 2 * TC_BLK;
   static constexpr int BYTES = BAR_OFF + 256;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr int H_COL = 256;  // two [128 x 128] H buffers at 256 and 384
+  static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
+// Fused SwiGLU apply on 2-SM tensor-core pairs (cta_group::2).  A cluster of two
+// CTAs owns a 256-token tile (128 per CTA) of one head; every MMA is M = 256:
+// A (queries, P) comes from each CTA's own rows, B (weights) is split in halves
+// between the two CTAs -- CTA 0 holds the W1 rows and CTA 1 the W3 rows of a
+// 64-wide m chunk for [H1 | H3], and each holds D/2 rows of W2 for O -- so each
+// CTA streams half the weight bytes per token.  The even CTA issues the MMAs;
+// both CTAs run TMA producers and epilogues, and the epilogues of both CTAs
+// report to the even CTA's barriers.
 template <int D>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmW,
@@ -412,128 +422,140 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nc = m / TC_MS;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-  uint64_t* qfull = bars + 0;
-  uint64_t* qfree = bars + 1;
-  uint64_t* wfull = bars + 2;   // [2]
-  uint64_t* wfree = bars + 4;   // [2]
-  uint64_t* hfull = bars + 6;   // [2]
-  uint64_t* hfree = bars + 8;   // [2]
-  uint64_t* pfull = bars + 10;  // [2]
-  uint64_t* pfree = bars + 12;  // [2]
-  uint64_t* odone = bars + 14;
-  uint64_t* ofree = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* qfull = bars + 0;   // leader: TMA bytes of both CTAs
+  uint64_t* qfree = bars + 1;   // both: MMA done reading Q
+  uint64_t* wfull = bars + 2;   // [NS] leader
+  uint64_t* wfree = wfull + L::NS;   // [NS] both
+  uint64_t* hfull = wfree + L::NS;   // [2] both
+  uint64_t* hfree = hfull + 2;       // [2] leader: 512 arrivals (both epilogues)
+  uint64_t* pfull = hfree + 2;       // [2] leader: 512 arrivals
+  uint64_t* pfree = pfull + 2;       // [2] both
+  uint64_t* odone = pfree + 2;       // both
+  uint64_t* ofree = odone + 1;       // leader: 512 arrivals
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ofree + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
     mbar_init(qfree, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < L::NS; ++i) {
       mbar_init(wfull + i, 1);
       mbar_init(wfree + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(hfull + i, 1);
-      mbar_init(hfree + i, 256);
-      mbar_init(pfull + i, 256);
+      mbar_init(hfree + i, 512);
+      mbar_init(pfull + i, 512);
       mbar_init(pfree + i, 1);
     }
     mbar_init(odone, 1);
-    mbar_init(ofree, 256);
+    mbar_init(ofree, 512);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{status, timeout_ns};
 
   if (warp == 0) {
     if (lane == 0) {
+      // ---------------- TMA producer (both CTAs): own Q rows, own half of each weight chunk
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmW);
       tma_prefetch_desc(&tmW2);
+      const uint32_t qfull_l = cluster_addr(qfull, 0);
       int gc = 0, it = 0;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++it) {
+      for (int item = pair; ok && item < n_items; item += npairs, ++it) {
         const int tile = item / H, h = item % H;
         if (it > 0 && !mbar_wait(qfree, (it - 1) & 1, g)) break;
-        mbar_expect_tx(qfull, L::KB * TC_BLK);
+        if (leader) mbar_expect_tx(qfull, 2 * L::KB * TC_BLK);
         for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_2d(smem + L::Q_OFF + kb * TC_BLK, &tmQ, qfull, h * D + kb * 64, tile * TC_TILE);
+          tma_load_2d_pair(smem + L::Q_OFF + kb * TC_BLK, &tmQ, qfull_l, h * D + kb * 64,
+                           tile * 2 * TC_TILE + (int)rank * TC_TILE);
         for (int c = 0; c < nc; ++c, ++gc) {
-          const int st = gc & 1;
-          if (gc >= 2 && !mbar_wait(wfree + st, ((gc >> 1) - 1) & 1, g)) { ok = false; break; }
+          const int st = gc % L::NS, use = gc / L::NS;
+          if (use > 0 && !mbar_wait(wfree + st, (use - 1) & 1, g)) { ok = false; break; }
           uint8_t* sw = smem + L::W_OFF + st * L::STAGE;
-          mbar_expect_tx(wfull + st, L::STAGE);
-          for (int kb = 0; kb < L::KB; ++kb) {
-            tma_load_2d(sw + kb * TC_BLK, &tmW, wfull + st, kb * 64, h * m + c * TC_MS);
-            tma_load_2d(sw + kb * TC_BLK + 8192, &tmW, wfull + st, kb * 64, H * m + h * m + c * TC_MS);
-          }
-          tma_load_2d(sw + L::W13_BYTES, &tmW2, wfull + st, c * TC_MS, h * D);
+          const uint32_t wfull_l = cluster_addr(wfull + st, 0);
+          if (leader) mbar_expect_tx(wfull + st, 2 * L::STAGE);
+          const int wrow = (rank == 0 ? 0 : H * m) + h * m + c * TC_MS;  // W1 rows (CTA 0) or W3 rows (CTA 1)
+          for (int kb = 0; kb < L::KB; ++kb) tma_load_2d_pair(sw + kb * 8192, &tmW, wfull_l, kb * 64, wrow);
+          tma_load_2d_pair(sw + L::W13_HALF, &tmW2, wfull_l, c * TC_MS, h * D + (int)rank * (D / 2));
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (even CTA only)
       const uint32_t sQ = smem_u32(smem + L::Q_OFF), sW = smem_u32(smem + L::W_OFF);
       const uint32_t sP = smem_u32(smem + L::P_OFF);
-      constexpr uint32_t ID_H = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t ID_O = idesc_bf16(128, D, false, false);
+      constexpr uint32_t ID_H = idesc_bf16(256, 128, false, false);
+      constexpr uint32_t ID_O = idesc_bf16(256, D, false, false);
       int gc = 0, it = 0;
       bool ok = true;
-      // O += P[g] W2c[g]^T for global chunk g (the chunk's W stage and P buffer are g & 1)
       auto do_o = [&](int gchunk, bool first_of_item) -> bool {
-        const int pb = gchunk & 1;
-        if (!mbar_wait(pfull + pb, (gchunk >> 1) & 1, g)) return false;
-        if (first_of_item && it > 0 && !mbar_wait(ofree, (it - 1) & 1, g)) return false;
+        const int pb = gchunk & 1, st = gchunk % L::NS;
+        if (!mbar_wait_cluster(pfull + pb, (gchunk >> 1) & 1, g)) return false;
+        if (first_of_item && it > 0 && !mbar_wait_cluster(ofree, (it - 1) & 1, g)) return false;
         tc_fence_after();
-        const uint32_t sw2 = sW + pb * L::STAGE + L::W13_BYTES;
+        const uint32_t sw2 = sW + st * L::STAGE + L::W13_HALF;
 #pragma unroll
         for (int kw = 0; kw < 4; ++kw)
-          umma_bf16_ss(tmem + 0, sdesc_sw128(sP + pb * TC_BLK + kw * 32, 16, 1024),
-                       sdesc_sw128(sw2 + kw * 32, 16, 1024), ID_O, (!first_of_item || kw > 0));
-        umma_commit(wfree + pb);
-        umma_commit(pfree + pb);
+          umma_bf16_pair(tmem + 0, sdesc_sw128(sP + pb * TC_BLK + kw * 32, 16, 1024),
+                         sdesc_sw128(sw2 + kw * 32, 16, 1024), ID_O, (!first_of_item || kw > 0));
+        umma_commit_pair(wfree + st);
+        umma_commit_pair(pfree + pb);
         return true;
       };
-      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++it) {
+      for (int item = pair; ok && item < n_items; item += npairs, ++it) {
         if (!mbar_wait(qfull, it & 1, g)) break;
         for (int c = 0; c < nc; ++c, ++gc) {
-          const int st = gc & 1;
-          if (!mbar_wait(wfull + st, (gc >> 1) & 1, g)) { ok = false; break; }
-          if (gc >= 2 && !mbar_wait(hfree + st, ((gc >> 1) - 1) & 1, g)) { ok = false; break; }
+          const int st = gc % L::NS, hb = gc & 1;
+          if (!mbar_wait(wfull + st, (gc / L::NS) & 1, g)) { ok = false; break; }
+          if (gc >= 2 && !mbar_wait_cluster(hfree + hb, ((gc >> 1) - 1) & 1, g)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sw = sW + st * L::STAGE;
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             const int kb = ks >> 2, kw = ks & 3;
-            umma_bf16_ss(tmem + L::H_COL + st * 128, sdesc_sw128(sQ + kb * TC_BLK + kw * 32, 16, 1024),
-                         sdesc_sw128(sw + kb * TC_BLK + kw * 32, 16, 1024), ID_H, ks > 0);
+            umma_bf16_pair(tmem + L::H_COL + hb * 128, sdesc_sw128(sQ + kb * TC_BLK + kw * 32, 16, 1024),
+                           sdesc_sw128(sw + kb * 8192 + kw * 32, 16, 1024), ID_H, ks > 0);
           }
-          umma_commit(hfull + st);
-          if (c == nc - 1) umma_commit(qfree);
+          umma_commit_pair(hfull + hb);
+          if (c == nc - 1) umma_commit_pair(qfree);
           if (c > 0 && !do_o(gc - 1, c - 1 == 0)) { ok = false; break; }
         }
         if (!ok) break;
         if (!do_o(gc - 1, nc == 1)) break;
-        umma_commit(odone);
+        umma_commit_pair(odone);
       }
     }
   } else {
+    // ---------------- epilogue warps 2..9 (both CTAs)
     const int q = warp & 3;
     const int ch = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const uint32_t hfree_l0 = cluster_addr(hfree, 0), hfree_l1 = cluster_addr(hfree + 1, 0);
+    const uint32_t pfull_l0 = cluster_addr(pfull, 0), pfull_l1 = cluster_addr(pfull + 1, 0);
+    const uint32_t ofree_l = cluster_addr(ofree, 0);
     int gc = 0, it = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++it) {
+    for (int item = pair; ok && item < n_items; item += npairs, ++it) {
       const int tile = item / H, h = item % H;
-      const int64_t t = (int64_t)tile * TC_TILE + row;
+      const int64_t t = (int64_t)tile * 2 * TC_TILE + (int64_t)rank * TC_TILE + row;
       const float r = (t < T) ? (rq ? rq[t * H + h] : 1.f) : 0.f;
       for (int c = 0; c < nc; ++c, ++gc) {
         const int hb = gc & 1;
@@ -545,27 +567,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tmem_ld_wait(a1);
         tmem_ld_wait(a3);
         tc_fence_before();
-        mbar_arrive(hfree + hb);
+        mbar_arrive_cluster(hb ? hfree_l1 : hfree_l0);
         uint32_t pk[16];
+        const float2 r2 = make_float2(r, r);
+        const float2 half2 = make_float2(0.5f, 0.5f);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          float o[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const float h1 = __uint_as_float(a1[j + k]) * r;
-            const float h3 = __uint_as_float(a3[j + k]) * r;
-            o[k] = h1 / (1.0f + __expf(-h1)) * h3;
-          }
-          pk[j >> 1] = pack_bf16x2(o[0], o[1]);
+          const float2 h1 = __fmul2_rn(make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1])), r2);
+          const float2 h3 = __fmul2_rn(make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1])), r2);
+          const float2 hh = __fmul2_rn(h1, half2);
+          const float2 th = make_float2(tanh_approx(hh.x), tanh_approx(hh.y));
+          const float2 sg = __ffma2_rn(th, half2, half2);
+          const float2 pv = __fmul2_rn(__fmul2_rn(h1, sg), h3);  // SiLU(h1) * h3
+          pk[j >> 1] = pack_bf16x2(pv.x, pv.y);
         }
-        if (gc >= 2 && !__all_sync(0xffffffffu, mbar_wait(pfree + hb, ((gc >> 1) - 1) & 1, g))) { ok = false; break; }
+        if (gc >= 2 && !__all_sync(0xffffffffu, mbar_wait(pfree + hb, ((gc >> 1) - 1) & 1, g))) {
+          ok = false;
+          break;
+        }
         uint8_t* sp = smem + L::P_OFF + hb * TC_BLK;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
           *reinterpret_cast<uint4*>(sp + sw128_offset(row, ch * 4 + cc)) =
               make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
         fence_async_smem();
-        mbar_arrive(pfull + hb);
+        mbar_arrive_cluster(hb ? pfull_l1 : pfull_l0);
       }
       if (!ok) break;
       if (!__all_sync(0xffffffffu, mbar_wait(odone, it & 1, g))) break;
@@ -589,15 +615,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(ofree);
+      mbar_arrive_cluster(ofree_l);
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 

@@ -396,26 +396,39 @@ int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t
               const ttt_dims& d, ttt_dtype dt, const Ws& w, cudaStream_t s) {
   if (T == 0) return TTT_OK;
   if (dt == TTT_BF16) {
-    const int tiles = (int)((T + TC_TILE - 1) / TC_TILE);
-    const int n_items = tiles * d.heads;
+    const int pair_tiles = (int)((T + 2 * TC_TILE - 1) / (2 * TC_TILE));
+    const int n_items = pair_tiles * d.heads;
     CUtensorMap tQ, tW, tW2;
     const uint64_t hd = (uint64_t)d.heads * d.d;
     if (!tmap_bf16(&tQ, Q, hd, (uint64_t)T, (uint64_t)ldq * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
     if (!tmap_bf16(&tW, w.wsh, (uint64_t)d.d, 3ull * d.heads * d.m, (uint64_t)d.d * 2, 64, 64)) return TTT_ERR_CUDA;
-    if (!tmap_bf16(&tW2, w.w2b, (uint64_t)d.m, (uint64_t)d.heads * d.d, (uint64_t)d.m * 2, 64, (uint32_t)d.d))
+    if (!tmap_bf16(&tW2, w.w2b, (uint64_t)d.m, (uint64_t)d.heads * d.d, (uint64_t)d.m * 2, 64, (uint32_t)d.d / 2))
       return TTT_ERR_CUDA;
-    const int grid = std::min(n_items, sm_count());
+    const int npairs = std::max(1, std::min(n_items, sm_count() / 2));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * npairs);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     ProfScope ps(TTT_PROF_APPLY, s);
+    __nv_bfloat16* Ob = (__nv_bfloat16*)O;
+    const unsigned long long to = wait_timeout_ns();
     if (d.d == 192) {
       auto k = k_apply_tc<192>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<192>::ALLOC));
-      k<<<grid, TC_THREADS, ApLayout<192>::ALLOC, s>>>(tQ, tW, tW2, rq, (__nv_bfloat16*)O, ldo, T, d.heads, d.m,
-                                                        n_items, w.status, wait_timeout_ns());
+      cfg.dynamicSmemBytes = ApLayout<192>::ALLOC;
+      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, rq, Ob, ldo, T, d.heads, d.m, n_items, w.status, to));
     } else {
       auto k = k_apply_tc<128>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<128>::ALLOC));
-      k<<<grid, TC_THREADS, ApLayout<128>::ALLOC, s>>>(tQ, tW, tW2, rq, (__nv_bfloat16*)O, ldo, T, d.heads, d.m,
-                                                        n_items, w.status, wait_timeout_ns());
+      cfg.dynamicSmemBytes = ApLayout<128>::ALLOC;
+      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, rq, Ob, ldo, T, d.heads, d.m, n_items, w.status, to));
     }
     TTT_LAUNCHED();
   } else {
