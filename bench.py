@@ -259,6 +259,7 @@ def run_ours(args, cfg):
     from test_weight_layers_b200 import build as B
     from test_weight_layers_b200 import synth as S
     from test_weight_layers_b200 import ttt as T
+    from test_weight_layers_b200.gcs import sharded_layer
 
     world, rank, local = dist_env()
     if world > 1:
@@ -323,15 +324,14 @@ def run_ours(args, cfg):
         elif world == 1:
             T.ttt_chunked(Wabi, Qx, Kx, Vuse, ex, Ox, Tn, cfg.chunk, 0, cfg.steps, ns, dm, io, ws)
         else:
-            chunk = cfg.chunk or Tn
-            for c0 in range(0, Tn, chunk):
-                c1 = min(Tn, c0 + chunk)
-                if cfg.chunk:
-                    T.ttt_apply(Wabi, Qx[c0:c1], Ox[c0:c1], c1 - c0, dm, io, ws)
-                for _ in range(cfg.steps):
-                    T.ttt_grad(Wabi, Kx[c0:c1], Vuse[c0:c1], ex[c0:c1], c1 - c0, dm, io, G, ws)
-                    dist.all_reduce(G)  # gradient of the whole (all-rank) chunk
-                    T.ttt_step(Wabi, G, ns, dm, T.TTT_BF16, ws)
+            sharded_layer(
+                Tn, cfg.steps,
+                grad=lambda t0, t1: (T.ttt_grad(Wabi, Kx[t0:t1], Vuse[t0:t1], ex[t0:t1], t1 - t0, dm, io, G, ws), G)[1],
+                allreduce=lambda g_: dist.all_reduce(g_),
+                step=lambda g_: T.ttt_step(Wabi, g_, ns, dm, T.TTT_BF16, ws),
+                apply=(lambda t0, t1: T.ttt_apply(Wabi, Qx[t0:t1], Ox[t0:t1], t1 - t0, dm, io, ws))
+                if cfg.chunk else None,
+                chunk=cfg.chunk, order=0)
             if not cfg.chunk:
                 T.ttt_apply(Wabi, Qx, Ox, Ta, dm, io, ws)
 

@@ -59,6 +59,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 // reductions of lane partials masked by head.
 
 constexpr int RN_MAX_VEC = 4;  // 16-byte vectors per lane: H*d <= 128 * VN elements
+constexpr int RN_TOKS = 4;     // tokens per warp iteration when only the norms are written
+constexpr int RN_TOK_VEC = 3;  // vectors per lane in that path: H*d <= 96 * VN elements
 
 template <typename T>
 __global__ void __launch_bounds__(256, 4) k_rownorm(T* X, int64_t ld, int64_t rows, int H, int d, float* r_out, int mode) {
@@ -92,6 +94,44 @@ __global__ void __launch_bounds__(256, 4) k_rownorm(T* X, int64_t ld, int64_t ro
             for (int i = 0; i < VN; ++i) x[i] *= inv;
             store16(row + h * d + v * VN, x);
           }
+        }
+      }
+    }
+    return;
+  }
+  if (mode == 0 && nvt <= 32 * RN_TOK_VEC) {
+    // norms only: four tokens per warp iteration, all their loads in flight together
+    for (int64_t t0 = warp_id * RN_TOKS; t0 < rows; t0 += nwarps * RN_TOKS) {
+      float ss[RN_TOKS][RN_TOK_VEC];
+      int hv[RN_TOK_VEC];
+#pragma unroll
+      for (int k = 0; k < RN_TOK_VEC; ++k) {
+        const int v = lane + 32 * k;
+        hv[k] = v < nvt ? v * VN / d : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < RN_TOKS; ++u) {
+        const int64_t t = t0 + u;
+#pragma unroll
+        for (int k = 0; k < RN_TOK_VEC; ++k) {
+          ss[u][k] = 0.f;
+          if (hv[k] >= 0 && t < rows) {
+            float x[VN];
+            load16(X + t * ld + (lane + 32 * k) * VN, x);
+#pragma unroll
+            for (int i = 0; i < VN; ++i) ss[u][k] = fmaf(x[i], x[i], ss[u][k]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < RN_TOKS; ++u) {
+        const int64_t t = t0 + u;
+        for (int h = 0; h < H; ++h) {
+          float p = 0.f;
+#pragma unroll
+          for (int k = 0; k < RN_TOK_VEC; ++k) p += (hv[k] == h) ? ss[u][k] : 0.f;
+          p = warp_sum(p);
+          if (lane == 0 && t < rows) r_out[t * H + h] = 1.0f / fmaxf(sqrtf(p), 1e-12f);
         }
       }
     }
@@ -145,90 +185,178 @@ __global__ void __launch_bounds__(256, 4) k_rownorm(T* X, int64_t ld, int64_t ro
 }
 
 // ---------------------------------------------------------------------------
+// Update-operand preparation: one pass over K and V that writes the fp16
+// operands of the tensor-core gradient kernel, K^ = k / max(||k||, 1e-12) per
+// head (or k itself) and V, densely [T][H*d].  bf16 -> fp16 is exact for values
+// in fp16's normal range; fp16 carries three more significand bits than bf16,
+// which the chained Muon updates need.  One warp per token, the whole row loaded
+// before any reduction.
+
+__device__ __forceinline__ void store16_h(__half* p, const float (&v)[8]) {
+  uint4 x;
+  x.x = pack_f16x2(v[0], v[1]);
+  x.y = pack_f16x2(v[2], v[3]);
+  x.z = pack_f16x2(v[4], v[5]);
+  x.w = pack_f16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = x;
+}
+
+__global__ void __launch_bounds__(256, 2) k_prep_kv(const __nv_bfloat16* __restrict__ K, int64_t ldk,
+                                                    const __nv_bfloat16* __restrict__ V, int64_t ldv,
+                                                    __half* __restrict__ Kh, __half* __restrict__ Vh, int64_t rows,
+                                                    int H, int d, int l2norm) {
+  constexpr int VN = 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int HD = H * d;
+  const int nvt = HD / VN;
+  for (int64_t t = warp_id; t < rows; t += nwarps) {
+    const __nv_bfloat16* krow = K + t * ldk;
+    const __nv_bfloat16* vrow = V + t * ldv;
+    if (nvt <= 32 * RN_MAX_VEC) {
+      float x[RN_MAX_VEC][VN], y[RN_MAX_VEC][VN];
+      int hv[RN_MAX_VEC];
+#pragma unroll
+      for (int k = 0; k < RN_MAX_VEC; ++k) {
+        const int v = lane + 32 * k;
+        hv[k] = v < nvt ? v * VN / d : -1;
+        if (hv[k] >= 0) {
+          load16(krow + v * VN, x[k]);
+          load16(vrow + v * VN, y[k]);
+        }
+      }
+      float inv[RN_MAX_VEC];
+#pragma unroll
+      for (int k = 0; k < RN_MAX_VEC; ++k) inv[k] = 1.f;
+      if (l2norm) {
+        float ss[RN_MAX_VEC];
+#pragma unroll
+        for (int k = 0; k < RN_MAX_VEC; ++k) {
+          ss[k] = 0.f;
+          if (hv[k] >= 0) {
+#pragma unroll
+            for (int i = 0; i < VN; ++i) ss[k] = fmaf(x[k][i], x[k][i], ss[k]);
+          }
+        }
+        for (int h = 0; h < H; ++h) {
+          float p = 0.f;
+#pragma unroll
+          for (int k = 0; k < RN_MAX_VEC; ++k) p += (hv[k] == h) ? ss[k] : 0.f;
+          p = warp_sum(p);
+          const float r = 1.0f / fmaxf(sqrtf(p), 1e-12f);
+#pragma unroll
+          for (int k = 0; k < RN_MAX_VEC; ++k)
+            if (hv[k] == h) inv[k] = r;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < RN_MAX_VEC; ++k)
+        if (hv[k] >= 0) {
+#pragma unroll
+          for (int i = 0; i < VN; ++i) x[k][i] *= inv[k];
+          store16_h(Kh + t * HD + (lane + 32 * k) * VN, x[k]);
+          store16_h(Vh + t * HD + (lane + 32 * k) * VN, y[k]);
+        }
+    } else {
+      for (int h = 0; h < H; ++h) {
+        float ss = 0.f;
+        for (int v = lane; v < d / VN; v += 32) {
+          float x[VN];
+          load16(krow + h * d + v * VN, x);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) ss = fmaf(x[i], x[i], ss);
+        }
+        ss = warp_sum(ss);
+        const float r = l2norm ? 1.0f / fmaxf(sqrtf(ss), 1e-12f) : 1.f;
+        for (int v = lane; v < d / VN; v += 32) {
+          float x[VN], y[VN];
+          load16(krow + h * d + v * VN, x);
+          load16(vrow + h * d + v * VN, y);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) x[i] *= r;
+          store16_h(Kh + t * HD + h * d + v * VN, x);
+          store16_h(Vh + t * HD + h * d + v * VN, y);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // ShortConv2D (VGG-T3 key design 2): depthwise 3x3 zero-padded cross-correlation
 // per frame on the (N, h, w, C) patch grid.  CTA = (frame, 64-channel group);
-// it slides down the frame keeping rows y-1, y, y+1 of its channels in shared
-// memory (with zero columns at x = -1 and x = w), so every input element is
-// read from HBM once.  threadIdx.x = 16-byte channel vector within the group,
-// threadIdx.y = x position (strided by blockDim.y).
+// threadIdx.x = 16-byte channel vector, threadIdx.y = x position (strided); the
+// CTA walks down the frame, so the three input rows an output row needs are
+// read from HBM once and re-served from L1 to the nine taps.
 
 constexpr int CONV_GROUP = 64;    // channels per CTA
-constexpr int CONV_MAX_W = 256;   // grid width limit of this kernel
+
+__device__ __forceinline__ void load16_nc(const float* p, float (&v)[4]) {
+  float4 x = __ldg(reinterpret_cast<const float4*>(p));
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void load16_nc(const __nv_bfloat16* p, float (&v)[8]) {
+  uint4 x = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_shortconv(const T* __restrict__ V, int64_t ldv, T* __restrict__ out, int64_t ldo,
                                                    const float* __restrict__ taps, int N, int gh, int gw, int C, int act) {
   constexpr int VN = Vec16<T>::N;
-  extern __shared__ float conv_sm[];   // [3][gw + 2][CONV_GROUP] fp32
   const int n = blockIdx.x;
   const int c0 = blockIdx.y * CONV_GROUP + threadIdx.x * VN;
-  const bool cvalid = c0 < C;
+  if (c0 >= C) return;
   float w[9][VN];
 #pragma unroll
   for (int i = 0; i < VN; ++i)
 #pragma unroll
-    for (int k = 0; k < 9; ++k) w[k][i] = cvalid ? taps[(c0 + i) * 9 + k] : 0.f;
-  const int W2 = gw + 2;
-  auto slot = [&](int r, int x) { return conv_sm + ((size_t)(r % 3) * W2 + (x + 1)) * CONV_GROUP + threadIdx.x * VN; };
-  // zero the padding columns of all three row slots and prefill rows -1 (zeros) and 0
-  for (int r = 0; r < 3; ++r)
-    if (threadIdx.y == 0) {
-#pragma unroll
-      for (int i = 0; i < VN; ++i) {
-        slot(r, -1)[i] = 0.f;
-        slot(r, gw)[i] = 0.f;
-      }
-    }
+    for (int k = 0; k < 9; ++k) w[k][i] = taps[(c0 + i) * 9 + k];
   const int64_t frame0 = (int64_t)n * gh * gw;
-  auto load_row = [&](int y) {  // row y into slot y % 3 (zeros outside the frame)
-    for (int x = threadIdx.y; x < gw; x += blockDim.y) {
-      float v[VN];
-      if (y >= 0 && y < gh && cvalid) {
-        load16(V + (frame0 + (int64_t)y * gw + x) * ldv + c0, v);
-      } else {
-#pragma unroll
-        for (int i = 0; i < VN; ++i) v[i] = 0.f;
-      }
-      float* dst = slot(y + 3, x);
-#pragma unroll
-      for (int i = 0; i < VN; ++i) dst[i] = v[i];
-    }
-  };
-  load_row(-1);
-  load_row(0);
   for (int y = 0; y < gh; ++y) {
-    load_row(y + 1);
-    __syncthreads();
     for (int x = threadIdx.y; x < gw; x += blockDim.y) {
       float acc[VN];
 #pragma unroll
       for (int i = 0; i < VN; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int dy = -1; dy <= 1; ++dy)
+      for (int dy = -1; dy <= 1; ++dy) {
+        const int yy = y + dy;
+        if (yy < 0 || yy >= gh) continue;
 #pragma unroll
         for (int dx = -1; dx <= 1; ++dx) {
-          const float* src = slot(y + dy + 3, x + dx);
+          const int xx = x + dx;
+          if (xx < 0 || xx >= gw) continue;
+          float v[VN];
+          load16_nc(V + (frame0 + (int64_t)yy * gw + xx) * ldv + c0, v);
           const int k = (dy + 1) * 3 + (dx + 1);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[k][i], src[i], acc[i]);
+          for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[k][i], v[i], acc[i]);
         }
+      }
       if (act == 1) {
 #pragma unroll
         for (int i = 0; i < VN; ++i) acc[i] = acc[i] / (1.0f + expf(-acc[i]));
       }
-      if (cvalid) store16(out + (frame0 + (int64_t)y * gw + x) * ldo + c0, acc);
+      store16(out + (frame0 + (int64_t)y * gw + x) * ldo + c0, acc);
     }
-    __syncthreads();
   }
 }
 
 // ---------------------------------------------------------------------------
-// bf16 shadows of the fp32 fast weights, laid out for the tensor-core kernels:
-//   Wsh rows [0, Hm): W1 [H][m][d];  [Hm, 2Hm): W3;  [2Hm, 3Hm): W2^T [H][m][d]
-//   W2b [H][d][m]  (W2 itself)
+// Low-precision copies of the fp32 fast weights, laid out for the tensor-core kernels:
+//   Wsh (bf16, apply) and Wsh16 (fp16, gradient) rows [0, Hm): W1 [H][m][d];
+//   [Hm, 2Hm): W3;  [2Hm, 3Hm): W2^T [H][m][d];   W2b [H][d][m] (bf16 W2, apply)
 
 __global__ void k_shadow(const float* __restrict__ W1, const float* __restrict__ W3, const float* __restrict__ W2,
-                         __nv_bfloat16* __restrict__ Wsh, __nv_bfloat16* __restrict__ W2b, int H, int d, int m) {
+                         __nv_bfloat16* __restrict__ Wsh, __nv_bfloat16* __restrict__ W2b, __half* __restrict__ Wsh16,
+                         int H, int d, int m) {
   const int64_t n = (int64_t)H * m * d;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     Wsh[i] = __float2bfloat16_rn(W1[i]);
@@ -237,8 +365,14 @@ __global__ void k_shadow(const float* __restrict__ W1, const float* __restrict__
     const int64_t h = i / ((int64_t)m * d);
     const int64_t rem = i % ((int64_t)m * d);
     const int64_t j = rem / d, k = rem % d;
-    Wsh[2 * n + i] = __float2bfloat16_rn(W2[(h * d + k) * m + j]);
+    const float w2t = W2[(h * d + k) * m + j];
+    Wsh[2 * n + i] = __float2bfloat16_rn(w2t);
     W2b[i] = __float2bfloat16_rn(W2[i]);
+    if (Wsh16) {  // fp16 copy only when a gradient kernel will read it
+      Wsh16[i] = __float2half_rn(W1[i]);
+      Wsh16[n + i] = __float2half_rn(W3[i]);
+      Wsh16[2 * n + i] = __float2half_rn(w2t);
+    }
   }
 }
 

@@ -60,6 +60,8 @@ struct UpdLayout {
 };
 
 constexpr int UPD_THREADS = 352;  // warp 0: forward TMA, 1: MMA, 2..9: epilogue, 10: backward TMA
+constexpr float GRAD_SCALE = 256.f;
+constexpr float GRAD_UNSCALE = 1.f / 256.f;
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
@@ -183,10 +185,10 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
       const uint32_t sW = smem_u32(smem + L::W_OFF), sF = smem_u32(smem + L::F_OFF);
       const uint32_t sB = smem_u32(smem + L::B_OFF), sDH = smem_u32(smem + L::DH_OFF);
       const uint32_t sU = smem_u32(smem + L::U_OFF);
-      constexpr uint32_t ID_F13 = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t ID_Z = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t ID_G13 = idesc_bf16(128, D, true, true);
-      constexpr uint32_t ID_G2 = idesc_bf16(128, 64, true, true);
+      constexpr uint32_t ID_F13 = idesc_f16(128, 128, false, false);
+      constexpr uint32_t ID_Z = idesc_f16(128, 64, false, false);
+      constexpr uint32_t ID_G13 = idesc_f16(128, D, true, true);
+      constexpr uint32_t ID_G2 = idesc_f16(128, 64, true, true);
       int fc = 0, bc = 0;
       // one forward block b of the current forward tile
       auto f_block = [&](int b) -> bool {
@@ -286,8 +288,10 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
       tc_fence_before();
       mbar_arrive(ffree);  // F may now be overwritten by the next tile's forward
       const float2 r2 = make_float2(r, r);
-      const float2 er2 = make_float2(-e * r, -e * r);   // -eta * r
-      const float2 ne2 = make_float2(-e, -e);
+      // dH and U~ are stored as fp16 scaled by 2^8 (clear of fp16 subnormals); the
+      // gradient readout multiplies by 2^-8, which is exact
+      const float2 er2 = make_float2(-e * r * GRAD_SCALE, -e * r * GRAD_SCALE);   // -eta * r
+      const float2 ne2 = make_float2(-e * GRAD_SCALE, -e * GRAD_SCALE);
       const float2 half2 = make_float2(0.5f, 0.5f);
       const float2 one2 = make_float2(1.f, 1.f);
       uint32_t p1[16], p3[16], pu[16];
@@ -307,9 +311,9 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
         const float2 d1 = __fmul2_rn(__fmul2_rn(dz, h3), qd);    // dL/dh1 (raw key)
         const float2 d3 = __fmul2_rn(dz, a);                     // dL/dh3 (raw key)
         const float2 ut = __fmul2_rn(ne2, u);                    // -eta u
-        p1[j >> 1] = pack_bf16x2(d1.x, d1.y);
-        p3[j >> 1] = pack_bf16x2(d3.x, d3.y);
-        pu[j >> 1] = pack_bf16x2(ut.x, ut.y);
+        p1[j >> 1] = pack_f16x2(d1.x, d1.y);
+        p3[j >> 1] = pack_f16x2(d3.x, d3.y);
+        pu[j >> 1] = pack_f16x2(ut.x, ut.y);
       }
       // dH / U~ buffer is free once the previous tile's backward has completed
       if (i > 0 && !__all_sync(0xffffffffu, mbar_wait(gdone, (i - 1) & 1, g))) { ok = false; break; }
@@ -354,8 +358,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(dst + c0 + j) =
-                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                            __uint_as_float(v[j + 3]));
+                make_float4(__uint_as_float(v[j]) * GRAD_UNSCALE, __uint_as_float(v[j + 1]) * GRAD_UNSCALE,
+                            __uint_as_float(v[j + 2]) * GRAD_UNSCALE, __uint_as_float(v[j + 3]) * GRAD_UNSCALE);
         }
       }
       // g2 columns of this slice: block rb holds d rows 64*rb .. 64*rb+127
@@ -370,8 +374,9 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
           float* dst = g2 + (int64_t)drow * m + slice * TC_MS + ch * 32;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                                              __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+            *reinterpret_cast<float4*>(dst + j) =
+                make_float4(__uint_as_float(v[j]) * GRAD_UNSCALE, __uint_as_float(v[j + 1]) * GRAD_UNSCALE,
+                            __uint_as_float(v[j + 2]) * GRAD_UNSCALE, __uint_as_float(v[j + 3]) * GRAD_UNSCALE);
         }
       }
     }

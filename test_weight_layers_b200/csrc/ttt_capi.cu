@@ -84,6 +84,9 @@ struct Ws {
   float* stepn;        // [3H][NORM_PARTS][2] partials of ||W||^2, ||W - lr D||^2
   float* rk;           // [T][H]
   float* rq;           // [T][H]
+  __half* wsh16;       // [3][H*m][d] fp16: W1, W3, W2^T (gradient kernel)
+  __half* kh16;        // [T][H*d] fp16 K^ (gradient kernel operand)
+  __half* vh16;        // [T][H*d] fp16 V
   size_t total;
   int s_max;
 };
@@ -129,6 +132,10 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_stepn = take(3 * H * NORM_PARTS * 2 * 4);
   const size_t o_rk = take((size_t)std::max<int64_t>(T, 1) * H * 4);
   const size_t o_rq = take((size_t)std::max<int64_t>(T, 1) * H * 4);
+  const bool tc = dt == TTT_BF16;
+  const size_t o_wsh16 = tc ? take(3 * n * 2) : 0;
+  const size_t o_kh = tc ? take((size_t)std::max<int64_t>(T, 1) * H * d * 2) : 0;
+  const size_t o_vh = tc ? take((size_t)std::max<int64_t>(T, 1) * H * d * 2) : 0;
   w.total = off;
   uint8_t* b = static_cast<uint8_t*>(base);
   if (b) {
@@ -145,6 +152,11 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
     w.stepn = reinterpret_cast<float*>(b + o_stepn);
     w.rk = reinterpret_cast<float*>(b + o_rk);
     w.rq = reinterpret_cast<float*>(b + o_rq);
+    if (tc) {
+      w.wsh16 = reinterpret_cast<__half*>(b + o_wsh16);
+      w.kh16 = reinterpret_cast<__half*>(b + o_kh);
+      w.vh16 = reinterpret_cast<__half*>(b + o_vh);
+    }
   }
   return w;
 }
@@ -193,14 +205,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D bf16 tensor [outer][inner] with row stride `row_bytes`, 128-byte swizzled boxes.
 bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-               uint32_t box_inner, uint32_t box_outer) {
+               uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  return fn(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -269,7 +282,7 @@ int launch_rownorm(T* X, int64_t ld, int64_t rows, const ttt_dims& d, float* r_o
   const int threads = 256;
   const int64_t warps = rows;
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((warps * 32 + threads - 1) / threads,
-                                                                   (int64_t)sm_count() * 16));
+                                                                   (int64_t)sm_count() * 8));
   ProfScope ps(TTT_PROF_NORM, s);
   k_rownorm<T><<<blocks, threads, 0, s>>>(X, ld, rows, d.heads, d.d, r_out, mode);
   TTT_LAUNCHED();
@@ -286,12 +299,51 @@ int launch_rownorm_any(const void* X, int64_t ld, int64_t rows, const ttt_dims& 
 int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStream_t s) {
   const int64_t n = (int64_t)d.heads * d.m * d.d;
   ProfScope ps(TTT_PROF_SHADOW, s);
-  k_shadow<<<grid1d(n, 256), 256, 0, s>>>(W.W1, W.W3, W.W2, w.wsh, w.w2b, d.heads, d.d, d.m);
+  k_shadow<<<grid1d(n, 256), 256, 0, s>>>(W.W1, W.W3, W.W2, w.wsh, w.w2b, w.wsh16, d.heads, d.d, d.m);
   TTT_LAUNCHED();
   return TTT_OK;
 }
 
-// gradient over T tokens -> G (fp32, [3][H*m*d]); shadow of W must be current (bf16)
+// fp16 gradient operands K^, V (dense [T][H*d]) from the caller's bf16 K, V
+int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, int64_t T, const ttt_dims& d, int l2norm,
+                   const Ws& w, cudaStream_t s) {
+  if (T == 0) return TTT_OK;
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 8));
+  ProfScope ps(TTT_PROF_NORM, s);
+  k_prep_kv<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, w.kh16, w.vh16, T,
+                                   d.heads, d.d, l2norm);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+struct UpdOperands {
+  const void* K;
+  int64_t ldk;
+  const void* V;
+  int64_t ldv;
+  const float* rk;
+};
+
+// Operands of the gradient kernels for T tokens: fp16 K^/V copies in bf16 mode,
+// the caller's K/V plus per-token inverse norms in fp32 mode.
+int prepare_update_operands(const void* K, int64_t ldk, const void* V, int64_t ldv, int64_t T, const ttt_dims& d,
+                            ttt_dtype dt, int l2norm, const Ws& w, cudaStream_t s, UpdOperands* op) {
+  if (dt == TTT_BF16) {
+    TTT_TRY(launch_prep_kv(K, ldk, V, ldv, T, d, l2norm, w, s));
+    const int64_t hd = (int64_t)d.heads * d.d;
+    *op = {w.kh16, hd, w.vh16, hd, nullptr};
+    return TTT_OK;
+  }
+  *op = {K, ldk, V, ldv, nullptr};
+  if (l2norm && T > 0) {
+    TTT_TRY(launch_rownorm_any(K, ldk, T, d, dt, w.rk, s));
+    op->rk = w.rk;
+  }
+  return TTT_OK;
+}
+
+// gradient over T tokens -> G (fp32, [3][H*m*d]); shadow of W must be current.
+// bf16 mode: K, V are the fp16 operands written by launch_prep_kv (ld = H*d, K^ normalised).
 int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta,
              const float* rk, int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, float* G, cudaStream_t s) {
   const int64_t n = (int64_t)d.heads * d.m * d.d;
@@ -306,11 +358,13 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
     S = std::max(1, std::min({sm_count() / std::max(1, slices * d.heads), w.s_max, tiles}));
     CUtensorMap tK, tV, tKb, tVb, tW;
     const uint64_t hd = (uint64_t)d.heads * d.d;
-    if (!tmap_bf16(&tK, K, hd, (uint64_t)T, (uint64_t)ldk * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
-    if (!tmap_bf16(&tV, V, hd, (uint64_t)T, (uint64_t)ldv * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
-    if (!tmap_bf16(&tKb, K, hd, (uint64_t)T, (uint64_t)ldk * 2, 64, UpdLayout<192>::BCH)) return TTT_ERR_CUDA;
-    if (!tmap_bf16(&tVb, V, hd, (uint64_t)T, (uint64_t)ldv * 2, 64, UpdLayout<192>::BCH)) return TTT_ERR_CUDA;
-    if (!tmap_bf16(&tW, w.wsh, (uint64_t)d.d, 3ull * d.heads * d.m, (uint64_t)d.d * 2, 64, 64)) return TTT_ERR_CUDA;
+    const CUtensorMapDataType F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!tmap_bf16(&tK, K, hd, (uint64_t)T, (uint64_t)ldk * 2, 64, TC_TILE, F16)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tV, V, hd, (uint64_t)T, (uint64_t)ldv * 2, 64, TC_TILE, F16)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tKb, K, hd, (uint64_t)T, (uint64_t)ldk * 2, 64, UpdLayout<192>::BCH, F16)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tVb, V, hd, (uint64_t)T, (uint64_t)ldv * 2, 64, UpdLayout<192>::BCH, F16)) return TTT_ERR_CUDA;
+    if (!tmap_bf16(&tW, w.wsh16, (uint64_t)d.d, 3ull * d.heads * d.m, (uint64_t)d.d * 2, 64, 64, F16))
+      return TTT_ERR_CUDA;
     dim3 grid(slices, d.heads, S);
     ProfScope ps(TTT_PROF_GRAD, s);
     if (d.d == 192) {
@@ -518,22 +572,17 @@ int ttt_shortconv2d(const void* V, int64_t ld_v, void* Vout, int64_t ld_out, con
   if (!V || !Vout || !taps || V == Vout) return TTT_ERR_INVALID;
   if (!aligned16(V) || !aligned16(Vout) || (ld_v * (int64_t)esize(dtype)) % 16 || (ld_out * (int64_t)esize(dtype)) % 16)
     return TTT_ERR_ALIGN;
-  if (w > CONV_MAX_W) return TTT_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
   const int vn = dtype == TTT_BF16 ? 8 : 4;
   const int gv = CONV_GROUP / vn;
   const dim3 block(gv, 256 / gv);
   const dim3 grid(N, (C + CONV_GROUP - 1) / CONV_GROUP);
-  const size_t smem = (size_t)3 * (w + 2) * CONV_GROUP * sizeof(float);
   ProfScope ps(TTT_PROF_CONV, s);
-  if (dtype == TTT_BF16) {
-    TTT_CHECK(cudaFuncSetAttribute(k_shortconv<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_shortconv<__nv_bfloat16><<<grid, block, smem, s>>>((const __nv_bfloat16*)V, ld_v, (__nv_bfloat16*)Vout, ld_out,
-                                                         taps, N, h, w, C, act);
-  } else {
-    TTT_CHECK(cudaFuncSetAttribute(k_shortconv<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    k_shortconv<float><<<grid, block, smem, s>>>((const float*)V, ld_v, (float*)Vout, ld_out, taps, N, h, w, C, act);
-  }
+  if (dtype == TTT_BF16)
+    k_shortconv<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)V, ld_v, (__nv_bfloat16*)Vout, ld_out, taps,
+                                                      N, h, w, C, act);
+  else
+    k_shortconv<float><<<grid, block, 0, s>>>((const float*)V, ld_v, (float*)Vout, ld_out, taps, N, h, w, C, act);
   TTT_LAUNCHED();
   return TTT_OK;
 }
@@ -551,13 +600,10 @@ int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int6
   if (T > 0 && !eta) return TTT_ERR_INVALID;
   cudaStream_t s = (cudaStream_t)stream;
   Ws w = carve(ws, dims, T, dtype);
-  const float* rk = nullptr;
-  if (io->qk_l2norm && T > 0) {
-    TTT_TRY(launch_rownorm_any(K, ldk, T, dims, dtype, w.rk, s));
-    rk = w.rk;
-  }
+  UpdOperands op;
+  TTT_TRY(prepare_update_operands(K, ldk, V, ldv, T, dims, dtype, io->qk_l2norm, w, s, &op));
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
-  return run_grad(W, K, ldk, V, ldv, eta, rk, T, dims, dtype, w, G, s);
+  return run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, T, dims, dtype, w, G, s);
 }
 
 int ttt_step(ttt_weights W, const float* G, const ttt_ns_cfg* ns, ttt_dims dims, ttt_dtype dtype, void* ws,
@@ -585,14 +631,11 @@ int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, in
   if (T == 0 || steps == 0) return TTT_OK;
   cudaStream_t s = (cudaStream_t)stream;
   Ws w = carve(ws, dims, T, dtype);
-  const float* rk = nullptr;
-  if (io->qk_l2norm) {
-    TTT_TRY(launch_rownorm_any(K, ldk, T, dims, dtype, w.rk, s));
-    rk = w.rk;
-  }
+  UpdOperands op;
+  TTT_TRY(prepare_update_operands(K, ldk, V, ldv, T, dims, dtype, io->qk_l2norm, w, s, &op));
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
   for (int st = 0; st < steps; ++st) {
-    TTT_TRY(run_grad(W, K, ldk, V, ldv, eta, rk, T, dims, dtype, w, w.G, s));
+    TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, T, dims, dtype, w, w.G, s));
     TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
   }
   return TTT_OK;
@@ -692,17 +735,16 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
     const uint8_t* v = static_cast<const uint8_t*>(V) + c0 * ldv * es;
     uint8_t* o = static_cast<uint8_t*>(O) + c0 * ldo * es;
     const float* e = eta + c0 * dims.heads;
-    const float* rk = nullptr;
     const float* rq = nullptr;
     if (io->qk_l2norm) {
-      TTT_TRY(launch_rownorm_any(k, ldk, tc, dims, dtype, w.rk, s));
       TTT_TRY(launch_rownorm_any(q, ldq, tc, dims, dtype, w.rq, s));
-      rk = w.rk;
       rq = w.rq;
     }
+    UpdOperands op;
+    TTT_TRY(prepare_update_operands(k, ldk, v, ldv, tc, dims, dtype, io->qk_l2norm, w, s, &op));
     if (order == 0) TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
     for (int st = 0; st < steps; ++st) {
-      TTT_TRY(run_grad(W, k, ldk, v, ldv, e, rk, tc, dims, dtype, w, w.G, s));
+      TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, e, op.rk, tc, dims, dtype, w, w.G, s));
       TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
     }
     if (order == 1) TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
