@@ -167,6 +167,14 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
                 int64_t T, int64_t chunk, int order, int steps, const ttt_ns_cfg* ns, ttt_dims dims,
                 const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
+/* Diagnostic for the timeout path: launches one single-warp kernel that waits on
+ * a barrier nothing ever signals, with a wait limit of `timeout_us`
+ * microseconds.  The wait gives up, records TTT_ERR_TIMEOUT in the workspace
+ * status word and the kernel returns, so the CUDA context stays usable; a
+ * following ttt_poll_status reports TTT_ERR_TIMEOUT until ttt_reset_status.
+ * timeout_us must be in [1, 10^7]. */
+int ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned timeout_us, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(int status);
 

@@ -285,10 +285,10 @@ __global__ void __launch_bounds__(256, 2) k_prep_kv(const __nv_bfloat16* __restr
 
 // ---------------------------------------------------------------------------
 // ShortConv2D (VGG-T3 key design 2): depthwise 3x3 zero-padded cross-correlation
-// per frame on the (N, h, w, C) patch grid.  CTA = (frame, 64-channel group);
-// threadIdx.x = 16-byte channel vector, threadIdx.y = x position (strided); the
-// CTA walks down the frame, so the three input rows an output row needs are
-// read from HBM once and re-served from L1 to the nine taps.
+// per frame on the (N, h, w, C) patch grid.  CTA = (frame, 64-channel group),
+// taps in shared memory; threadIdx.x = 16-byte channel vector, threadIdx.y walks
+// the frame's tokens, so a token's neighbours are read from HBM once and
+// re-served from L1 to the nine taps.
 
 constexpr int CONV_GROUP = 64;    // channels per CTA
 
@@ -308,44 +308,53 @@ __device__ __forceinline__ void load16_nc(const __nv_bfloat16* p, float (&v)[8])
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) k_shortconv(const T* __restrict__ V, int64_t ldv, T* __restrict__ out, int64_t ldo,
-                                                   const float* __restrict__ taps, int N, int gh, int gw, int C, int act) {
+__global__ void __launch_bounds__(256, 4) k_shortconv(const T* __restrict__ V, int64_t ldv, T* __restrict__ out,
+                                                      int64_t ldo, const float* __restrict__ taps, int N, int gh,
+                                                      int gw, int C, int act) {
   constexpr int VN = Vec16<T>::N;
-  const int n = blockIdx.x;
-  const int c0 = blockIdx.y * CONV_GROUP + threadIdx.x * VN;
+  __shared__ __align__(16) float wt[9][CONV_GROUP];  // this CTA's taps, [tap][channel]
+  const int n = blockIdx.x, g0 = blockIdx.y * CONV_GROUP;
+  const int nthr = blockDim.x * blockDim.y, tid = threadIdx.y * blockDim.x + threadIdx.x;
+  for (int i = tid; i < 9 * CONV_GROUP; i += nthr) {
+    const int k = i / CONV_GROUP, c = i % CONV_GROUP;
+    wt[k][c] = (g0 + c < C) ? taps[(g0 + c) * 9 + k] : 0.f;
+  }
+  __syncthreads();
+  const int c0 = g0 + threadIdx.x * VN;
   if (c0 >= C) return;
-  float w[9][VN];
-#pragma unroll
-  for (int i = 0; i < VN; ++i)
-#pragma unroll
-    for (int k = 0; k < 9; ++k) w[k][i] = taps[(c0 + i) * 9 + k];
   const int64_t frame0 = (int64_t)n * gh * gw;
-  for (int y = 0; y < gh; ++y) {
-    for (int x = threadIdx.y; x < gw; x += blockDim.y) {
-      float acc[VN];
+  const int ntok = gh * gw;
+  for (int p = threadIdx.y; p < ntok; p += blockDim.y) {
+    const int y = p / gw, x = p % gw;
+    float acc[VN];
 #pragma unroll
-      for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int dy = -1; dy <= 1; ++dy) {
-        const int yy = y + dy;
-        if (yy < 0 || yy >= gh) continue;
+    for (int dy = -1; dy <= 1; ++dy) {
+      const int yy = y + dy;
+      if (yy < 0 || yy >= gh) continue;
 #pragma unroll
-        for (int dx = -1; dx <= 1; ++dx) {
-          const int xx = x + dx;
-          if (xx < 0 || xx >= gw) continue;
-          float v[VN];
-          load16_nc(V + (frame0 + (int64_t)yy * gw + xx) * ldv + c0, v);
-          const int k = (dy + 1) * 3 + (dx + 1);
+      for (int dx = -1; dx <= 1; ++dx) {
+        const int xx = x + dx;
+        if (xx < 0 || xx >= gw) continue;
+        float v[VN];
+        load16_nc(V + (frame0 + (int64_t)yy * gw + xx) * ldv + c0, v);
+        const float* wk = &wt[(dy + 1) * 3 + (dx + 1)][threadIdx.x * VN];
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[k][i], v[i], acc[i]);
+        for (int i = 0; i < VN; i += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(wk + i);
+          acc[i] = fmaf(w4.x, v[i], acc[i]);
+          acc[i + 1] = fmaf(w4.y, v[i + 1], acc[i + 1]);
+          acc[i + 2] = fmaf(w4.z, v[i + 2], acc[i + 2]);
+          acc[i + 3] = fmaf(w4.w, v[i + 3], acc[i + 3]);
         }
       }
-      if (act == 1) {
-#pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = acc[i] / (1.0f + expf(-acc[i]));
-      }
-      store16(out + (frame0 + (int64_t)y * gw + x) * ldo + c0, acc);
     }
+    if (act == 1) {
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[i] = acc[i] / (1.0f + expf(-acc[i]));
+    }
+    store16(out + (frame0 + p) * ldo + c0, acc);
   }
 }
 
@@ -817,6 +826,21 @@ __global__ void __launch_bounds__(256) k_apply_f32(const float* __restrict__ Q, 
       if (t0 + t < T) O[(t0 + t) * ldo + (int64_t)h * d + kk] = acc[q];
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Timeout-path diagnostic: wait on a barrier that is initialised for one arrival
+// that never comes.  The bounded wait records DEV_TIMEOUT and the kernel returns.
+__global__ void k_selftest_wait(unsigned int* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const Guard g{status, timeout_ns};
+  const bool ok = mbar_wait(&bar, 0, g);
+  (void)__all_sync(0xffffffffu, ok);
 }
 
 }  // namespace ttt

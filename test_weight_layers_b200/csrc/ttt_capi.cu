@@ -752,6 +752,15 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
   return TTT_OK;
 }
 
+int ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned timeout_us, void* stream) {
+  if (!ws || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTT_ERR_WORKSPACE;
+  if (timeout_us < 1 || timeout_us > 10000000u) return TTT_ERR_INVALID;
+  k_selftest_wait<<<1, 32, 0, (cudaStream_t)stream>>>(static_cast<unsigned int*>(ws),
+                                                       (unsigned long long)timeout_us * 1000ull);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
 const char* ttt_status_string(int status) {
   switch (status) {
     case TTT_OK: return "ok";

@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
             "ttt_chunked": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), Dims,
                                 ctypes.POINTER(IOCfg), I, P, SZ, P]),
             "ttt_status_string": (ctypes.c_char_p, [I]),
+            "ttt_selftest_wait_timeout": (I, [P, SZ, ctypes.c_uint, P]),
             "ttt_launch_count": (ctypes.c_uint64, []),
             "ttt_profile_enable": (I, [I]),
             "ttt_profile_reset": (I, []),
@@ -185,6 +186,11 @@ def ttt_chunked(W: Weights, Q, K, V, eta, O, T, chunk, order, steps, ns: NSCfg, 
     _check("ttt_chunked", lib().ttt_chunked(W, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(O), T, chunk, order, steps,
                                             ctypes.byref(ns), dm, ctypes.byref(io), dtype_code(Q.dtype), _ptr(ws),
                                             ws.numel(), _stream(stream)))
+
+
+def ttt_selftest_wait_timeout(ws, timeout_us: int, stream=None):
+    _check("ttt_selftest_wait_timeout", lib().ttt_selftest_wait_timeout(_ptr(ws), ws.numel(), timeout_us,
+                                                                        _stream(stream)))
 
 
 def ttt_launch_count() -> int:

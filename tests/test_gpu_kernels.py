@@ -175,3 +175,22 @@ def test_update_eta_zero_keeps_weights_bf16():
     T.ttt_update(W.abi, K, V, eta, T_, 1, T.ns_cfg(), dm, T.io_cfg(), ws)
     check_status(ws)
     assert max(weight_errors(W.oracle(), before)) < 1e-6
+
+
+def test_device_wait_timeout_is_reported_and_context_survives():
+    # a wait on a barrier nothing signals gives up after its limit, records the
+    # timeout in the status word and returns; the context keeps working afterwards
+    dm = T.dims(1, 128, 64)
+    ws = T.workspace(dm, 256, T.TTT_BF16)
+    T.ttt_reset_status(ws)
+    assert T.ttt_poll_status(ws) == T.TTT_OK
+    T.ttt_selftest_wait_timeout(ws, 50_000)
+    assert T.ttt_poll_status(ws) == T.TTT_ERR_TIMEOUT
+    T.ttt_reset_status(ws)
+    assert T.ttt_poll_status(ws) == T.TTT_OK
+    W = DevWeights(*rand_weights(1, 128, 64, 60))
+    Q = rand_tokens(256, 1, 128, torch.bfloat16, 61).cuda()
+    O_ = torch.zeros_like(Q)
+    T.ttt_apply(W.abi, Q, O_, 256, dm, T.io_cfg(), ws)
+    check_status(ws)
+    assert rel_fro(f64(O_), O.apply(W.oracle(), f64(Q))) < 1e-2
