@@ -581,6 +581,94 @@ __global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const flo
     }
 }
 
+// Gram matrices A_b = X_b X_b^T for the Newton-Schulz batch: upper-triangular
+// 64x64 tiles only (A is symmetric), split-K over NS_GRAM_SPLIT slices of the
+// long dimension for parallelism.  grid (tiles, NS_GRAM_SPLIT, batch); partial
+// P[s][b][i][j] for the tile's (i, j); k_gram_reduce sums the slices in fixed
+// order and mirrors the lower triangle.
+constexpr int NS_GRAM_SPLIT = 4;
+
+__global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float* __restrict__ X, int64_t sX,
+                                                      float* __restrict__ P) {
+  __shared__ __align__(16) float As[2][16][64];
+  __shared__ __align__(16) float Bs[2][16][64];
+  const int rt = (r + 63) / 64;
+  // tile index -> (ti <= tj) in row-major upper-triangular order
+  int t = blockIdx.x, ti = 0;
+  while (t >= rt - ti) { t -= rt - ti; ++ti; }
+  const int tj = ti + t;
+  const int s = blockIdx.y, b = blockIdx.z;
+  const int kper = ((c + NS_GRAM_SPLIT - 1) / NS_GRAM_SPLIT + 15) / 16 * 16;
+  const int k_begin = s * kper, k_end = min(c, k_begin + kper);
+  const float* x = X + (int64_t)b * sX;
+  const int m0 = ti * 64, n0 = tj * 64;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  float ra[4], rb[4];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = tid + 256 * q, kk = i & 15, mm = i >> 4, gk = k0 + kk;
+      ra[q] = (m0 + mm < r && gk < k_end) ? x[(int64_t)(m0 + mm) * c + gk] : 0.f;
+      rb[q] = (n0 + mm < r && gk < k_end) ? x[(int64_t)(n0 + mm) * c + gk] : 0.f;
+    }
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = tid + 256 * q;
+      As[buf][i & 15][i >> 4] = ra[q];
+      Bs[buf][i & 15][i >> 4] = rb[q];
+    }
+  };
+  float acc[4][4] = {};
+  int buf = 0;
+  if (k_begin < k_end) {
+    load(k_begin);
+    stash(0);
+  }
+  __syncthreads();
+  for (int k0 = k_begin; k0 < k_end; k0 += 16) {
+    const bool more = k0 + 16 < k_end;
+    if (more) load(k0 + 16);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float a4[4] = {av.x, av.y, av.z, av.w};
+      const float b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+    }
+    if (more) stash(buf ^ 1);
+    __syncthreads();
+    buf ^= 1;
+  }
+  float* out = P + ((int64_t)s * gridDim.z + b) * (int64_t)r * r;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
+      if (gm < r && gn < r) out[(int64_t)gm * r + gn] = acc[i][j];
+    }
+}
+
+// A[b][i][j] = sum_s P[s][b][min(i,j)][max(i,j)] (slices in fixed order)
+__global__ void k_gram_reduce(int r, int nb, const float* __restrict__ P, float* __restrict__ A) {
+  const int64_t n = (int64_t)r * r;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * nb; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t b = e / n, ij = e % n;
+    const int i = (int)(ij / r), j = (int)(ij % r);
+    const int64_t src = b * n + (int64_t)min(i, j) * r + max(i, j);
+    float acc = 0.f;
+#pragma unroll
+    for (int s = 0; s < NS_GRAM_SPLIT; ++s) acc += P[(int64_t)s * nb * n + src];
+    A[e] = acc;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Muon weight step (ZipMap key design 3): W <- ||W|| (W - lr D) / ||W - lr D||,
 // D in W's orientation (k_ns_finish), or G itself when Newton-Schulz is off.

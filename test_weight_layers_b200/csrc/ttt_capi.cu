@@ -80,6 +80,7 @@ struct Ws {
   float* X2;           // [3H][m*d]
   float* A;            // [3H][r*r]
   float* B;            // [3H][r*r]
+  float* gram;         // [NS_GRAM_SPLIT][3H][r*r] split-K partials of the Gram matrices
   float* norms;        // [3H][NORM_PARTS] partial sums of squares of G
   float* stepn;        // [3H][NORM_PARTS][2] partials of ||W||^2, ||W - lr D||^2
   float* rk;           // [T][H]
@@ -128,6 +129,7 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_X2 = take(3 * n * 4);
   const size_t o_A = take(3 * H * r * r * 4);
   const size_t o_B = take(3 * H * r * r * 4);
+  const size_t o_gram = take((size_t)NS_GRAM_SPLIT * 3 * H * r * r * 4);
   const size_t o_norms = take(3 * H * NORM_PARTS * 4);
   const size_t o_stepn = take(3 * H * NORM_PARTS * 2 * 4);
   const size_t o_rk = take((size_t)std::max<int64_t>(T, 1) * H * 4);
@@ -148,6 +150,7 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
     w.X2 = reinterpret_cast<float*>(b + o_X2);
     w.A = reinterpret_cast<float*>(b + o_A);
     w.B = reinterpret_cast<float*>(b + o_B);
+    w.gram = reinterpret_cast<float*>(b + o_gram);
     w.norms = reinterpret_cast<float*>(b + o_norms);
     w.stepn = reinterpret_cast<float*>(b + o_stepn);
     w.rk = reinterpret_cast<float*>(b + o_rk);
@@ -415,8 +418,9 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
     float* X2 = w.X2;
     const int rt = (r + 63) / 64, ct = (c + 63) / 64;
     for (int it = 0; it < ns.iters; ++it) {
-      k_gemm_f32<true><<<dim3(rt, rt, nb), 256, 0, s>>>(r, r, c, X, c, n, X, c, n, w.A, r, (int64_t)r * r, nullptr,
-                                                         1.f, 0.f);
+      k_gram_partial<<<dim3(rt * (rt + 1) / 2, NS_GRAM_SPLIT, nb), 256, 0, s>>>(r, c, X, n, w.gram);
+      TTT_LAUNCHED();
+      k_gram_reduce<<<grid1d((int64_t)nb * r * r, 256), 256, 0, s>>>(r, nb, w.gram, w.A);
       TTT_LAUNCHED();
       k_gemm_f32<false><<<dim3(rt, rt, nb), 256, 0, s>>>(r, r, r, w.A, r, (int64_t)r * r, w.A, r, (int64_t)r * r, w.B,
                                                           r, (int64_t)r * r, w.A, ns.c, ns.b);
