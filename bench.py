@@ -7,8 +7,9 @@ One step is one pass of the whole layer over the workload's tokens, starting
 from the initial fast weights: [ShortConv2D on V] + L2-normalised update
 (gradient over every token, Newton-Schulz, norm-preserving step; twice for the
 two-step workload; per chunk for the streaming workload) + apply.  Inputs are
-seeded synthetic tensors already resident in HBM; they are larger than L2, so
-no flush is needed between steps.  With N > 1 (torchrun, one rank per GPU)
+seeded synthetic tensors already resident in HBM; at the large workloads they
+are larger than L2, so no flush is needed between steps; smaller workloads
+overwrite a buffer larger than L2 before every step, outside its events.  With N > 1 (torchrun, one rank per GPU)
 each rank holds its own token shard of one N-times-larger layer and the
 per-step gradient is summed over ranks with an NCCL all-reduce before the
 Muon step (the pages' global context synchronisation); per-GPU work is fixed,
@@ -35,6 +36,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "TTT-layer tokens/sec (update+apply) and % of B200 bf16 tensor peak"
 UNIT = "tokens/s"
+L2_BYTES = 126 << 20
+L2_FLUSH_BYTES = 512 << 20
 
 
 def parse():
@@ -210,7 +213,7 @@ def run_reference(args, cfg):
     line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(cfg, args.gpus),
+            "config": workload_config(cfg, args.gpus, "host-side oracle; no GPU caches involved"),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": f"each step: fp64 oracle on {sample} of {cfg.tokens} tokens (gradient, "
                                        f"Newton-Schulz step, apply), extrapolated linearly in tokens"},
@@ -222,7 +225,7 @@ def run_reference(args, cfg):
 # ---------------------------------------------------------------------------- GPU arm
 
 
-def workload_config(cfg, n):
+def workload_config(cfg, n, l2_note):
     return {"workload": (f"{cfg.name}: {cfg.frames} frames x ({cfg.grid_h}x{cfg.grid_w}+{cfg.special}) = "
                          f"{cfg.tokens} tokens per GPU, {cfg.heads} heads d={cfg.d} m={cfg.m}, {cfg.steps} Muon "
                          f"step(s){', ShortConv2D on V' if cfg.conv else ''}"
@@ -230,7 +233,7 @@ def workload_config(cfg, n):
                          f"apply on {cfg.apply_tokens} tokens"),
             "tokens_per_gpu": cfg.tokens, "heads": cfg.heads, "d": cfg.d, "m": cfg.m, "inner_steps": cfg.steps,
             "chunk": cfg.chunk or None, "qk_l2norm": True,
-            "l2": "inputs larger than L2 (126 MB), no flush between steps",
+            "l2": l2_note,
             "parallelism": "single GPU" if n == 1 else f"token-sharded x{n}, NCCL all-reduce of the gradient"}
 
 
@@ -281,17 +284,20 @@ def run_ours(args, cfg):
     g = torch.Generator(device=dev)
     g.manual_seed(cfg.seed * 1000 + rank)
 
-    def randn_bf16(rows, cols):
-        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+    tdt = cfg.torch_dtype
+    dcode = T.dtype_code(tdt)
+
+    def randn_rows(rows, cols):
+        out = torch.empty((rows, cols), dtype=tdt, device=dev)
         step = 1 << 17
         for r0 in range(0, rows, step):
             r1 = min(rows, r0 + step)
-            out[r0:r1] = torch.randn((r1 - r0, cols), generator=g, device=dev).to(torch.bfloat16)
+            out[r0:r1] = torch.randn((r1 - r0, cols), generator=g, device=dev).to(tdt)
         return out
 
-    K = randn_bf16(Tn, D)
-    V = randn_bf16(Tn, D)
-    Q = randn_bf16(Ta, D)
+    K = randn_rows(Tn, D)
+    V = randn_rows(Tn, D)
+    Q = randn_rows(Ta, D)
     if cfg.eta_kind == "linear":
         w_eta = torch.randn((cfg.model_dim, H), generator=g, device=dev) / math.sqrt(cfg.model_dim)
         eta = torch.empty((Tn, H), dtype=torch.float32, device=dev)
@@ -306,9 +312,9 @@ def run_ours(args, cfg):
     Wabi = T.weights(*W)
     taps = S.conv_taps(cfg.seed, D).to(dev) if cfg.conv else None
     Vc = torch.empty_like(V) if cfg.conv else None
-    O = torch.empty((Ta, D), dtype=torch.bfloat16, device=dev)
+    O = torch.empty((Ta, D), dtype=tdt, device=dev)
     G = torch.empty(3 * H * m * d, dtype=torch.float32, device=dev)
-    ws = T.workspace(dm, cfg.chunk or max(Tn, Ta), T.TTT_BF16, device=dev)
+    ws = T.workspace(dm, cfg.chunk or max(Tn, Ta), dcode, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def layer(Kx, Vx, Qx, ex, Ox):
@@ -328,7 +334,7 @@ def run_ours(args, cfg):
                 Tn, cfg.steps,
                 grad=lambda t0, t1: (T.ttt_grad(Wabi, Kx[t0:t1], Vuse[t0:t1], ex[t0:t1], t1 - t0, dm, io, G, ws), G)[1],
                 allreduce=lambda g_: dist.all_reduce(g_),
-                step=lambda g_: T.ttt_step(Wabi, g_, ns, dm, T.TTT_BF16, ws),
+                step=lambda g_: T.ttt_step(Wabi, g_, ns, dm, dcode, ws),
                 apply=(lambda t0, t1: T.ttt_apply(Wabi, Qx[t0:t1], Ox[t0:t1], t1 - t0, dm, io, ws))
                 if cfg.chunk else None,
                 chunk=cfg.chunk, order=0)
@@ -339,6 +345,8 @@ def run_ours(args, cfg):
         if world > 1:
             dist.barrier(device_ids=[local])
 
+    resident = sum(x.numel() * x.element_size() for x in (K, V, Q, eta, O))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if resident < 2 * L2_BYTES else None
     for _ in range(args.warmup):
         layer(K, V, Q, eta, O)
     torch.cuda.synchronize(dev)
@@ -352,17 +360,30 @@ def run_ours(args, cfg):
     clocks = ClockSampler(bus_id_of(dev))
     time.sleep(0.3)  # let the sampler start
     launches0 = T.ttt_launch_count()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        layer(K, V, Q, eta, O)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            layer(K, V, Q, eta, O)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / args.steps
+    else:
+        # inputs fit in L2: overwrite a buffer larger than L2 before every step and
+        # time each step on its own events, so the flush is outside the timed steps
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            flush.fill_(1)
+            a.record(stream)
+            layer(K, V, Q, eta, O)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
     launches = T.ttt_launch_count() - launches0
     clk = clocks.stop()
     barrier()
     T.ttt_profile_enable(False)
-    ms = e0.elapsed_time(e1) / args.steps
     if world > 1:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -381,19 +402,31 @@ def run_ours(args, cfg):
     tok_per_launch = Tn if not cfg.chunk else cfg.chunk
     grad_flops = 12.0 * H * d * m * tok_per_launch
     roof = None
-    if g_n:
+    if g_n and dcode == T.TTT_BF16:
         ach = grad_flops / (g_ms / g_n / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
                 "traffic": traffic_per_launch(tok_per_launch), "kernel": "k_update_grad_tc",
-                "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
+                "peak_kind": f"fp16/bf16 dense (same tensor rate), sustained, {peaks['source']}",
+                "launch_ms": g_ms / g_n}
+    elif g_n:
+        # fp32 mode: CUDA-core FMA pipe, 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz
+        ach = grad_flops / (g_ms / g_n / 1e3) / 1e12
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roof = {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": None, "kernel": "k_grad_f32", "peak_kind": "fp32 FMA, derived from unit counts and max clock",
                 "launch_ms": g_ms / g_n}
     kernels = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps} for k, v in prof.items()}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(cfg, world),
+            "vs_baseline": None, "dtype": "bf16" if dcode == T.TTT_BF16 else "f32", "data": "synthetic",
+            "config": workload_config(cfg, world, "inputs larger than L2 (126 MB), no flush between steps"
+                                      if flush is None else
+                                      f"inputs fit in L2: {L2_FLUSH_BYTES >> 20} MB written before every step, "
+                                      "outside its events"),
             "tflops": tflops, "frac_of_bf16_peak": tflops * 1e12 / world / (peaks["bf16_tflops_sustained"] * 1e12),
+            "update_operands": "fp16 (exact from bf16 inputs)" if dcode == T.TTT_BF16 else "fp32",
             "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clk}
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
