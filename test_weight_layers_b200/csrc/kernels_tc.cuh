@@ -76,7 +76,9 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // drains F_i from TMEM into registers first and releases it, so F_(i+1) runs
 // while the epilogue computes; G_i is interleaved with F_(i+1) once the
 // epilogue has written dH_i.  K and V are read twice from L2 (once per ring),
-// which buys the latency hiding that a single resident tile cannot.
+// which buys the latency hiding that a single resident tile cannot.  The MMA
+// issue loop is straight-line code (compile-time block indices) run by a whole
+// converged warp with one elected lane issuing.
 template <int D>
 __global__ void __launch_bounds__(UPD_THREADS, 1)
     k_update_grad_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -180,86 +182,112 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      const uint32_t sW = smem_u32(smem + L::W_OFF), sF = smem_u32(smem + L::F_OFF);
-      const uint32_t sB = smem_u32(smem + L::B_OFF), sDH = smem_u32(smem + L::DH_OFF);
-      const uint32_t sU = smem_u32(smem + L::U_OFF);
+    {  // ---------------- MMA issuer: the whole warp runs the loop and waits,
+       // the elected lane issues the MMAs and commits
+      const bool leader = elect_one();
+      // Base descriptors; an operand at byte offset o from a base is the base
+      // descriptor + o/16 (the address field holds addr/16 and every operand
+      // lies below 256 KB, so the add never carries out of the field).
+      const uint64_t dW = sdesc_sw128(smem_u32(smem + L::W_OFF), 16, 1024);
+      const uint64_t dF = sdesc_sw128(smem_u32(smem + L::F_OFF), 16, 1024);
+      const uint64_t dB = sdesc_sw128(smem_u32(smem + L::B_OFF), L::BCHUNK, 1024);
+      const uint64_t dDH = sdesc_sw128(smem_u32(smem + L::DH_OFF), TC_BLK, 1024);
+      const uint64_t dU = sdesc_sw128(smem_u32(smem + L::U_OFF), TC_BLK, 1024);
       constexpr uint32_t ID_F13 = idesc_f16(128, 128, false, false);
       constexpr uint32_t ID_Z = idesc_f16(128, 64, false, false);
       constexpr uint32_t ID_G13 = idesc_f16(128, D, true, true);
       constexpr uint32_t ID_G2 = idesc_f16(128, 64, true, true);
-      int fc = 0, bc = 0;
-      // one forward block b of the current forward tile
-      auto f_block = [&](int b) -> bool {
-        const int st = fc % L::NF, use = fc / L::NF;
-        if (!mbar_wait(ffull + st, use & 1, g)) return false;
+      uint32_t fst = 0, fph = 0, bst = 0, bph = 0;  // ring stage and phase parity
+      bool ok = true;
+      // forward block b (compile-time) of the current forward tile
+      auto F = [&](auto bc) {
+        constexpr int b = decltype(bc)::value;
+        ok &= __all_sync(0xffffffffu, mbar_wait(ffull + fst, fph, g));
         tc_fence_after();
-        const uint32_t a0 = sF + st * TC_BLK;
-        if (b < L::KB) {
+        const uint64_t a0 = dF + (uint64_t)(fst * (TC_BLK >> 4));
+        if (leader) {
+          if constexpr (b < L::KB) {
 #pragma unroll
-          for (int kw = 0; kw < 4; ++kw)
-            umma_bf16_ss(tmem + 0, sdesc_sw128(a0 + kw * 32, 16, 1024),
-                         sdesc_sw128(sW + b * L::W_BLK + kw * 32, 16, 1024), ID_F13, (b > 0 || kw > 0));
-        } else {
-          const int vb = b - L::KB;
+            for (int kw = 0; kw < 4; ++kw)
+              umma_bf16_ss(tmem + 0, a0 + kw * 2, dW + (b * L::W_BLK + kw * 32) / 16, ID_F13,
+                           (b > 0 || kw > 0) ? 1u : 0u);
+          } else {
 #pragma unroll
-          for (int kw = 0; kw < 4; ++kw)
-            umma_bf16_ss(tmem + 128, sdesc_sw128(a0 + kw * 32, 16, 1024),
-                         sdesc_sw128(sW + vb * L::W_BLK + 16384 + kw * 32, 16, 1024), ID_Z, (vb > 0 || kw > 0));
-        }
-        umma_commit(fempty + st);
-        ++fc;
-        return true;
-      };
-      // one backward chunk c of tile i (dH/U~ of tile i must be in shared memory)
-      auto g_chunk = [&](int i, int c) -> bool {
-        const int st = bc % L::NB, use = bc / L::NB;
-        if (!mbar_wait(bfull + st, use & 1, g)) return false;
-        tc_fence_after();
-        const uint32_t b0 = sB + st * L::BSTAGE;
-#pragma unroll
-        for (int j = 0; j < L::BCH / 16; ++j) {
-          const int ks = c * (L::BCH / 16) + j;
-          const uint32_t acc = (i > 0 || ks > 0);
-          umma_bf16_ss(tmem + L::G13_COL, sdesc_sw128(sDH + ks * 2048, TC_BLK, 1024),
-                       sdesc_sw128(b0 + j * 2048, L::BCHUNK, 1024), ID_G13, acc);
-#pragma unroll
-          for (int rb = 0; rb < L::N_G2; ++rb)
-            umma_bf16_ss(tmem + L::G2_COL + rb * 64,
-                         sdesc_sw128(b0 + (L::KB + rb) * L::BCHUNK + j * 2048, L::BCHUNK, 1024),
-                         sdesc_sw128(sU + ks * 2048, TC_BLK, 1024), ID_G2, acc);
-        }
-        umma_commit(bempty + st);
-        ++bc;
-        return true;
-      };
-      bool ok = mbar_wait(wfull, 0, g);
-      if (ok && ntiles > 0) {
-        for (int b = 0; ok && b < L::NFB; ++b) ok = f_block(b);
-        if (ok) umma_commit(fdone);
-      }
-      for (int i = 0; ok && i < ntiles; ++i) {
-        const bool has_next = i + 1 < ntiles;
-        // F_(i+1) may overwrite TMEM F once the epilogue has drained F_i
-        if (has_next && !mbar_wait(ffree, i & 1, g)) break;
-        // the first forward blocks cover the epilogue's compute, then F and G alternate
-        int fb = 0, gcn = 0;
-        const int lead = has_next ? (L::NFB < 3 ? L::NFB : 3) : 0;
-        for (; ok && fb < lead; ++fb) ok = f_block(fb);
-        if (!ok) break;
-        if (has_next && fb == L::NFB) umma_commit(fdone);
-        if (!mbar_wait(edone, i & 1, g)) break;
-        tc_fence_after();
-        while (ok && (gcn < L::NBC || (has_next && fb < L::NFB))) {
-          if (gcn < L::NBC) ok = g_chunk(i, gcn++);
-          if (ok && has_next && fb < L::NFB) {
-            ok = f_block(fb++);
-            if (ok && fb == L::NFB) umma_commit(fdone);
+            for (int kw = 0; kw < 4; ++kw)
+              umma_bf16_ss(tmem + 128, a0 + kw * 2, dW + ((b - L::KB) * L::W_BLK + 16384 + kw * 32) / 16, ID_Z,
+                           (b > L::KB || kw > 0) ? 1u : 0u);
           }
+          umma_commit(fempty + fst);
         }
-        if (!ok) break;
-        umma_commit(gdone);
+        __syncwarp();
+        fph ^= (fst == L::NF - 1) ? 1u : 0u;
+        fst = (fst == L::NF - 1) ? 0u : fst + 1;
+      };
+      // backward chunk c (compile-time) of the current backward tile; acc0 = 0
+      // only for the very first gradient MMA of the token range
+      auto G = [&](auto cc, uint32_t acc0) {
+        constexpr int c = decltype(cc)::value;
+        ok &= __all_sync(0xffffffffu, mbar_wait(bfull + bst, bph, g));
+        tc_fence_after();
+        const uint64_t b0 = dB + (uint64_t)(bst * (L::BSTAGE >> 4));
+        if (leader) {
+#pragma unroll
+          for (int j = 0; j < L::BCH / 16; ++j) {
+            const int ks = c * (L::BCH / 16) + j;
+            const uint32_t acc = (c == 0 && j == 0) ? acc0 : 1u;
+            umma_bf16_ss(tmem + L::G13_COL, dDH + ks * 128, b0 + j * 128, ID_G13, acc);
+#pragma unroll
+            for (int rb = 0; rb < L::N_G2; ++rb)
+              umma_bf16_ss(tmem + L::G2_COL + rb * 64, b0 + ((L::KB + rb) * L::BCHUNK + j * 2048) / 16,
+                           dU + ks * 128, ID_G2, acc);
+          }
+          umma_commit(bempty + bst);
+        }
+        __syncwarp();
+        bph ^= (bst == L::NB - 1) ? 1u : 0u;
+        bst = (bst == L::NB - 1) ? 0u : bst + 1;
+      };
+      ok = __all_sync(0xffffffffu, mbar_wait(wfull, 0, g));
+      if (ok && ntiles > 0) {
+        static_for<0, L::NFB>(F);
+        if (leader) umma_commit(fdone);
+        __syncwarp();
+      }
+      // forward blocks issued before the backward: they cover the epilogue's
+      // compute; then G_i and the rest of F_(i+1) alternate so both TMA rings
+      // stay busy (issuing F_(i+1) whole drains the forward ring: slower)
+      constexpr int LEAD = L::NFB < 3 ? L::NFB : 3;
+      constexpr int NSTEP = (L::NBC > L::NFB - LEAD) ? L::NBC : L::NFB - LEAD;
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const uint32_t acc0 = i > 0 ? 1u : 0u;
+        if (i + 1 < ntiles) {
+          // F_(i+1) may overwrite TMEM F once the epilogue has drained F_i
+          ok &= __all_sync(0xffffffffu, mbar_wait(ffree, i & 1, g));
+          static_for<0, LEAD>(F);
+          if constexpr (LEAD == L::NFB) {
+            if (leader) umma_commit(fdone);
+            __syncwarp();
+          }
+          ok &= __all_sync(0xffffffffu, mbar_wait(edone, i & 1, g));
+          tc_fence_after();
+          static_for<0, NSTEP>([&](auto kc) {
+            constexpr int k = decltype(kc)::value;
+            if constexpr (k < L::NBC) G(kc, acc0);
+            if constexpr (LEAD + k < L::NFB) {
+              F(std::integral_constant<int, LEAD + k>{});
+              if constexpr (LEAD + k + 1 == L::NFB) {
+                if (leader) umma_commit(fdone);
+                __syncwarp();
+              }
+            }
+          });
+        } else {
+          ok &= __all_sync(0xffffffffu, mbar_wait(edone, i & 1, g));
+          tc_fence_after();
+          static_for<0, L::NBC>([&](auto kc) { G(kc, acc0); });
+        }
+        if (leader) umma_commit(gdone);
+        __syncwarp();
       }
     }
   } else {
@@ -286,7 +314,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
       tmem_ld_wait(a3);
       tmem_ld_wait(az);
       tc_fence_before();
-      mbar_arrive(ffree);  // F may now be overwritten by the next tile's forward
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(ffree, 32);  // F may now be overwritten by the next tile's forward
       const float2 r2 = make_float2(r, r);
       // dH and U~ are stored as fp16 scaled by 2^8 (clear of fp16 subnormals); the
       // gradient readout multiplies by 2^-8, which is exact
@@ -328,7 +357,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
         *reinterpret_cast<uint4*>(su + off) = make_uint4(pu[4 * c], pu[4 * c + 1], pu[4 * c + 2], pu[4 * c + 3]);
       }
       fence_async_smem();
-      mbar_arrive(edone);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(edone, 32);
     }
     if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(gdone, (ntiles - 1) & 1, g));
     if (ok && ntiles == 0) {
@@ -398,27 +428,35 @@ struct ApLayout {
   static constexpr int Q_OFF = 0;                        // this CTA's 128 query tokens, all d
   static constexpr int W13_HALF = KB * 64 * 128;         // this CTA's 64 rows of [W1c; W3c] (W1c or W3c)
   static constexpr int W2_HALF = (D / 2) * 128;          // this CTA's D/2 rows of W2c (64 m each)
-  static constexpr int STAGE = W13_HALF + W2_HALF;
-  static constexpr int NS = 3;                           // weight ring stages
-  static constexpr int W_OFF = Q_OFF + KB * TC_BLK;
-  static constexpr int P_OFF = W_OFF + NS * STAGE;
+  static constexpr int NS13 = 4;                         // W1|W3 ring stages (freed after the H MMAs)
+  static constexpr int NS2 = 4;                          // W2 ring stages (freed after the O MMAs)
+  static constexpr int W13_OFF = Q_OFF + KB * TC_BLK;
+  static constexpr int W2_OFF = W13_OFF + NS13 * W13_HALF;
+  static constexpr int P_OFF = W2_OFF + NS2 * W2_HALF;
   static constexpr int BAR_OFF = P_OFF + 2 * TC_BLK;
   static constexpr int BYTES = BAR_OFF + 256;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr int H_COL = 256;  // two [128 x 128] H buffers at 256 and 384
   static_assert(ALLOC <= 232448, "shared memory budget");
+  static_assert(2 * 2 + 2 * NS13 + 2 * NS2 + 4 * 2 + 2 <= 31, "barrier budget");
 };
+
+constexpr int AP_THREADS = 352;  // warp 0: Q + W1|W3 TMA, 1: MMA, 2..9: epilogue, 10: W2 TMA
 
 // Fused SwiGLU apply on 2-SM tensor-core pairs (cta_group::2).  A cluster of two
 // CTAs owns a 256-token tile (128 per CTA) of one head; every MMA is M = 256:
 // A (queries, P) comes from each CTA's own rows, B (weights) is split in halves
 // between the two CTAs -- CTA 0 holds the W1 rows and CTA 1 the W3 rows of a
 // 64-wide m chunk for [H1 | H3], and each holds D/2 rows of W2 for O -- so each
-// CTA streams half the weight bytes per token.  The even CTA issues the MMAs;
-// both CTAs run TMA producers and epilogues, and the epilogues of both CTAs
-// report to the even CTA's barriers.
+// CTA streams half the weight bytes per token.  W1|W3 and W2 stream through
+// separate rings with their own producers: a W1|W3 stage is free as soon as its
+// H MMAs complete, while W2 of chunk c is consumed only after H of chunk c+1
+// (one ring would hold every stage across two chunks and leave the chunk
+// period bound by the L2 round trip).  The even CTA issues the MMAs; both CTAs
+// run TMA producers and epilogues, and the epilogues of both CTAs report to the
+// even CTA's barriers.
 template <int D>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(AP_THREADS, 1)
     k_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmW,
                const __grid_constant__ CUtensorMap tmW2, const float* __restrict__ rq, __nv_bfloat16* __restrict__ O,
                int64_t ldo, int64_t T, int H, int m, int n_items, unsigned int* status,
@@ -433,24 +471,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int nc = m / TC_MS;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-  uint64_t* qfull = bars + 0;   // leader: TMA bytes of both CTAs
-  uint64_t* qfree = bars + 1;   // both: MMA done reading Q
-  uint64_t* wfull = bars + 2;   // [NS] leader
-  uint64_t* wfree = wfull + L::NS;   // [NS] both
-  uint64_t* hfull = wfree + L::NS;   // [2] both
-  uint64_t* hfree = hfull + 2;       // [2] leader: 512 arrivals (both epilogues)
-  uint64_t* pfull = hfree + 2;       // [2] leader: 512 arrivals
-  uint64_t* pfree = pfull + 2;       // [2] both
-  uint64_t* odone = pfree + 2;       // both
-  uint64_t* ofree = odone + 1;       // leader: 512 arrivals
+  uint64_t* qfull = bars + 0;              // leader: TMA bytes of both CTAs
+  uint64_t* qfree = bars + 1;              // both: MMA done reading Q
+  uint64_t* w13full = bars + 2;            // [NS13] leader
+  uint64_t* w13free = w13full + L::NS13;   // [NS13] both
+  uint64_t* w2full = w13free + L::NS13;    // [NS2] leader
+  uint64_t* w2free = w2full + L::NS2;      // [NS2] both
+  uint64_t* hfull = w2free + L::NS2;       // [2] both
+  uint64_t* hfree = hfull + 2;             // [2] leader: 512 arrivals (both epilogues)
+  uint64_t* pfull = hfree + 2;             // [2] leader: 512 arrivals
+  uint64_t* pfree = pfull + 2;             // [2] both
+  uint64_t* odone = pfree + 2;             // both
+  uint64_t* ofree = odone + 1;             // leader: 512 arrivals
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ofree + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
     mbar_init(qfree, 1);
-    for (int i = 0; i < L::NS; ++i) {
-      mbar_init(wfull + i, 1);
-      mbar_init(wfree + i, 1);
+    for (int i = 0; i < L::NS13; ++i) {
+      mbar_init(w13full + i, 1);
+      mbar_init(w13free + i, 1);
+    }
+    for (int i = 0; i < L::NS2; ++i) {
+      mbar_init(w2full + i, 1);
+      mbar_init(w2free + i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(hfull + i, 1);
@@ -475,10 +519,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer (both CTAs): own Q rows, own half of each weight chunk
+      // ---------------- Q + W1|W3 producer (both CTAs): own Q rows, own half of each [W1c; W3c]
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmW);
-      tma_prefetch_desc(&tmW2);
       const uint32_t qfull_l = cluster_addr(qfull, 0);
       int gc = 0, it = 0;
       bool ok = true;
@@ -490,61 +533,100 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tma_load_2d_pair(smem + L::Q_OFF + kb * TC_BLK, &tmQ, qfull_l, h * D + kb * 64,
                            tile * 2 * TC_TILE + (int)rank * TC_TILE);
         for (int c = 0; c < nc; ++c, ++gc) {
-          const int st = gc % L::NS, use = gc / L::NS;
-          if (use > 0 && !mbar_wait(wfree + st, (use - 1) & 1, g)) { ok = false; break; }
-          uint8_t* sw = smem + L::W_OFF + st * L::STAGE;
-          const uint32_t wfull_l = cluster_addr(wfull + st, 0);
-          if (leader) mbar_expect_tx(wfull + st, 2 * L::STAGE);
+          const int st = gc % L::NS13, use = gc / L::NS13;
+          if (use > 0 && !mbar_wait(w13free + st, (use - 1) & 1, g)) { ok = false; break; }
+          uint8_t* sw = smem + L::W13_OFF + st * L::W13_HALF;
+          const uint32_t full_l = cluster_addr(w13full + st, 0);
+          if (leader) mbar_expect_tx(w13full + st, 2 * L::W13_HALF);
           const int wrow = (rank == 0 ? 0 : H * m) + h * m + c * TC_MS;  // W1 rows (CTA 0) or W3 rows (CTA 1)
-          for (int kb = 0; kb < L::KB; ++kb) tma_load_2d_pair(sw + kb * 8192, &tmW, wfull_l, kb * 64, wrow);
-          tma_load_2d_pair(sw + L::W13_HALF, &tmW2, wfull_l, c * TC_MS, h * D + (int)rank * (D / 2));
+          for (int kb = 0; kb < L::KB; ++kb) tma_load_2d_pair(sw + kb * 8192, &tmW, full_l, kb * 64, wrow);
+        }
+      }
+    }
+  } else if (warp == 10) {
+    if (lane == 0) {
+      // ---------------- W2 producer (both CTAs): own D/2 rows of each W2 chunk
+      tma_prefetch_desc(&tmW2);
+      int gc = 0;
+      bool ok = true;
+      for (int item = pair; ok && item < n_items; item += npairs) {
+        const int h = item % H;
+        for (int c = 0; c < nc; ++c, ++gc) {
+          const int st = gc % L::NS2, use = gc / L::NS2;
+          if (use > 0 && !mbar_wait(w2free + st, (use - 1) & 1, g)) { ok = false; break; }
+          const uint32_t full_l = cluster_addr(w2full + st, 0);
+          if (leader) mbar_expect_tx(w2full + st, 2 * L::W2_HALF);
+          tma_load_2d_pair(smem + L::W2_OFF + st * L::W2_HALF, &tmW2, full_l, c * TC_MS,
+                           h * D + (int)rank * (D / 2));
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      // ---------------- MMA issuer (even CTA only)
-      const uint32_t sQ = smem_u32(smem + L::Q_OFF), sW = smem_u32(smem + L::W_OFF);
-      const uint32_t sP = smem_u32(smem + L::P_OFF);
+    if (leader) {
+      // ---------------- MMA issuer (even CTA only): the whole warp runs the loop
+      // and waits, the elected lane issues
+      const bool el = elect_one();
+      const uint64_t dQ = sdesc_sw128(smem_u32(smem + L::Q_OFF), 16, 1024);
+      const uint64_t dW13 = sdesc_sw128(smem_u32(smem + L::W13_OFF), 16, 1024);
+      const uint64_t dW2 = sdesc_sw128(smem_u32(smem + L::W2_OFF), 16, 1024);
+      const uint64_t dP = sdesc_sw128(smem_u32(smem + L::P_OFF), 16, 1024);
       constexpr uint32_t ID_H = idesc_bf16(256, 128, false, false);
       constexpr uint32_t ID_O = idesc_bf16(256, D, false, false);
-      int gc = 0, it = 0;
-      bool ok = true;
-      auto do_o = [&](int gchunk, bool first_of_item) -> bool {
-        const int pb = gchunk & 1, st = gchunk % L::NS;
-        if (!mbar_wait_cluster(pfull + pb, (gchunk >> 1) & 1, g)) return false;
-        if (first_of_item && it > 0 && !mbar_wait_cluster(ofree, (it - 1) & 1, g)) return false;
+      uint32_t s13 = 0, p13 = 0;  // W1|W3 ring stage and parity
+      uint32_t s2 = 0, p2 = 0;    // W2 ring stage and parity (of the next O chunk)
+      // O += P_c W2_c for the previous chunk (global chunk index gcp)
+      auto do_o = [&](uint32_t gcp, bool first_of_item, int it) -> bool {
+        const uint32_t pb = gcp & 1;
+        bool w = mbar_wait(w2full + s2, p2, g) && mbar_wait_cluster(pfull + pb, (gcp >> 1) & 1, g);
+        if (first_of_item && it > 0) w = w && mbar_wait_cluster(ofree, (it - 1) & 1, g);
+        if (!__all_sync(0xffffffffu, w)) return false;
         tc_fence_after();
-        const uint32_t sw2 = sW + st * L::STAGE + L::W13_HALF;
+        if (el) {
+          const uint64_t a0 = dP + pb * (TC_BLK >> 4);
+          const uint64_t b0 = dW2 + s2 * (L::W2_HALF >> 4);
 #pragma unroll
-        for (int kw = 0; kw < 4; ++kw)
-          umma_bf16_pair(tmem + 0, sdesc_sw128(sP + pb * TC_BLK + kw * 32, 16, 1024),
-                         sdesc_sw128(sw2 + kw * 32, 16, 1024), ID_O, (!first_of_item || kw > 0));
-        umma_commit_pair(wfree + st);
-        umma_commit_pair(pfree + pb);
+          for (int kw = 0; kw < 4; ++kw)
+            umma_bf16_pair(tmem + 0, a0 + kw * 2, b0 + kw * 2, ID_O, (!first_of_item || kw > 0) ? 1u : 0u);
+          umma_commit_pair(w2free + s2);
+          umma_commit_pair(pfree + pb);
+        }
+        __syncwarp();
+        p2 ^= (s2 == L::NS2 - 1) ? 1u : 0u;
+        s2 = (s2 == L::NS2 - 1) ? 0u : s2 + 1;
         return true;
       };
+      uint32_t gc = 0;  // global chunk counter (H buffer gc & 1)
+      int it = 0;
+      bool ok = true;
       for (int item = pair; ok && item < n_items; item += npairs, ++it) {
-        if (!mbar_wait(qfull, it & 1, g)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(qfull, it & 1, g))) break;
         for (int c = 0; c < nc; ++c, ++gc) {
-          const int st = gc % L::NS, hb = gc & 1;
-          if (!mbar_wait(wfull + st, (gc / L::NS) & 1, g)) { ok = false; break; }
-          if (gc >= 2 && !mbar_wait_cluster(hfree + hb, ((gc >> 1) - 1) & 1, g)) { ok = false; break; }
+          const uint32_t hb = gc & 1;
+          bool w = mbar_wait(w13full + s13, p13, g);
+          if (gc >= 2) w = w && mbar_wait_cluster(hfree + hb, ((gc >> 1) - 1) & 1, g);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sw = sW + st * L::STAGE;
+          if (el) {
+            const uint64_t b0 = dW13 + s13 * (L::W13_HALF >> 4);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const int kb = ks >> 2, kw = ks & 3;
-            umma_bf16_pair(tmem + L::H_COL + hb * 128, sdesc_sw128(sQ + kb * TC_BLK + kw * 32, 16, 1024),
-                           sdesc_sw128(sw + kb * 8192 + kw * 32, 16, 1024), ID_H, ks > 0);
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const int kb = ks >> 2, kw = ks & 3;
+              umma_bf16_pair(tmem + L::H_COL + hb * 128, dQ + (kb * TC_BLK + kw * 32) / 16,
+                             b0 + (kb * 8192 + kw * 32) / 16, ID_H, ks > 0 ? 1u : 0u);
+            }
+            umma_commit_pair(w13free + s13);
+            umma_commit_pair(hfull + hb);
+            if (c == nc - 1) umma_commit_pair(qfree);
           }
-          umma_commit_pair(hfull + hb);
-          if (c == nc - 1) umma_commit_pair(qfree);
-          if (c > 0 && !do_o(gc - 1, c - 1 == 0)) { ok = false; break; }
+          __syncwarp();
+          p13 ^= (s13 == L::NS13 - 1) ? 1u : 0u;
+          s13 = (s13 == L::NS13 - 1) ? 0u : s13 + 1;
+          if (c > 0 && !do_o(gc - 1, c == 1, it)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!do_o(gc - 1, nc == 1)) break;
-        umma_commit_pair(odone);
+        if (!do_o(gc - 1, nc == 1, it)) break;
+        if (el) umma_commit_pair(odone);
+        __syncwarp();
       }
     }
   } else {
@@ -572,7 +654,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tmem_ld_wait(a1);
         tmem_ld_wait(a3);
         tc_fence_before();
-        mbar_arrive_cluster(hb ? hfree_l1 : hfree_l0);
+        warp_arrive_cluster(hb ? hfree_l1 : hfree_l0);
         uint32_t pk[16];
         const float2 r2 = make_float2(r, r);
         const float2 half2 = make_float2(0.5f, 0.5f);
@@ -596,7 +678,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           *reinterpret_cast<uint4*>(sp + sw128_offset(row, ch * 4 + cc)) =
               make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
         fence_async_smem();
-        mbar_arrive_cluster(hb ? pfull_l1 : pfull_l0);
+        warp_arrive_cluster(hb ? pfull_l1 : pfull_l0);
       }
       if (!ok) break;
       if (!__all_sync(0xffffffffu, mbar_wait(odone, it & 1, g))) break;
@@ -620,7 +702,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive_cluster(ofree_l);
+      warp_arrive_cluster(ofree_l);
     }
   }
 

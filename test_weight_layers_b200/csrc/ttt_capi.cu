@@ -470,7 +470,7 @@ int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * npairs);
-    cfg.blockDim = dim3(TC_THREADS);
+    cfg.blockDim = dim3(AP_THREADS);
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
