@@ -428,12 +428,14 @@ struct ApLayout {
   static constexpr int Q_OFF = 0;                        // this CTA's 128 query tokens, all d
   static constexpr int W13_HALF = KB * 64 * 128;         // this CTA's 64 rows of [W1c; W3c] (W1c or W3c)
   static constexpr int W2_HALF = (D / 2) * 128;          // this CTA's D/2 rows of W2c (64 m each)
-  static constexpr int NS13 = 4;                         // W1|W3 ring stages (freed after the H MMAs)
+  static constexpr int NS13 = 3;                         // W1|W3 ring stages (freed after the H MMAs)
   static constexpr int NS2 = 4;                          // W2 ring stages (freed after the O MMAs)
   static constexpr int W13_OFF = Q_OFF + KB * TC_BLK;
   static constexpr int W2_OFF = W13_OFF + NS13 * W13_HALF;
   static constexpr int P_OFF = W2_OFF + NS2 * W2_HALF;
-  static constexpr int BAR_OFF = P_OFF + 2 * TC_BLK;
+  static constexpr int OST = 32 * 64;                    // per epilogue warp: [32 rows x 32 cols] bf16 staging
+  static constexpr int OST_OFF = P_OFF + 2 * TC_BLK;     // 8 warps' staging tiles (64-byte swizzle)
+  static constexpr int BAR_OFF = OST_OFF + 8 * OST;
   static constexpr int BYTES = BAR_OFF + 256;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr int H_COL = 256;  // two [128 x 128] H buffers at 256 and 384
@@ -458,8 +460,8 @@ constexpr int AP_THREADS = 352;  // warp 0: Q + W1|W3 TMA, 1: MMA, 2..9: epilogu
 template <int D>
 __global__ void __launch_bounds__(AP_THREADS, 1)
     k_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmW,
-               const __grid_constant__ CUtensorMap tmW2, const float* __restrict__ rq, __nv_bfloat16* __restrict__ O,
-               int64_t ldo, int64_t T, int H, int m, int n_items, unsigned int* status,
+               const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmO,
+               const float* __restrict__ rq, int64_t T, int H, int m, int n_items, unsigned int* status,
                unsigned long long timeout_ns) {
   using L = ApLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -658,12 +660,14 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
         uint32_t pk[16];
         const float2 r2 = make_float2(r, r);
         const float2 half2 = make_float2(0.5f, 0.5f);
+        // sigmoid(h1) = 1/2 + tanh(h1/2)/2 with tanh in half precision (two per
+        // MUFU operation): its error (~2^-11) is well below the bf16 rounding of P
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float2 h1 = __fmul2_rn(make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1])), r2);
           const float2 h3 = __fmul2_rn(make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1])), r2);
           const float2 hh = __fmul2_rn(h1, half2);
-          const float2 th = make_float2(tanh_approx(hh.x), tanh_approx(hh.y));
+          const float2 th = unpack_f16x2(tanh_f16x2(pack_f16x2(hh.x, hh.y)));
           const float2 sg = __ffma2_rn(th, half2, half2);
           const float2 pv = __fmul2_rn(__fmul2_rn(h1, sg), h3);  // SiLU(h1) * h3
           pk[j >> 1] = pack_bf16x2(pv.x, pv.y);
@@ -683,27 +687,44 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
       if (!ok) break;
       if (!__all_sync(0xffffffffu, mbar_wait(odone, it & 1, g))) break;
       tc_fence_after();
-      __nv_bfloat16* orow = O + t * ldo + (int64_t)h * D;
+      // O readout: this warp's 32 token rows x D/2 columns; all TMEM loads first,
+      // then O is released to the next item's MMAs while the stores proceed
+      constexpr int NP = D / 64;  // 32-column pieces per warp
+      uint32_t ov[NP][32];
 #pragma unroll
-      for (int c0 = ch * (D / 2); c0 < (ch + 1) * (D / 2); c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + c0, v);
-        tmem_ld_wait(v);
-        if (t < T) {
+      for (int p = 0; p < NP; ++p) tmem_ld32(tmem + lane_base + ch * (D / 2) + p * 32, ov[p]);
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint4 x;
-            x.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-            x.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-            x.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
-            x.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
-            *reinterpret_cast<uint4*>(orow + c0 + j) = x;
-          }
-        }
-      }
+      for (int p = 0; p < NP; ++p) tmem_ld_wait(ov[p]);
       tc_fence_before();
       warp_arrive_cluster(ofree_l);
+      // each piece goes through this warp's swizzled staging tile and a TMA store
+      // (rows past T are clipped by the tensor map)
+      uint8_t* stg = smem + L::OST_OFF + (warp - 2) * L::OST;
+      const int orow0 = tile * 2 * TC_TILE + (int)rank * TC_TILE + q * 32;
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        if (p > 0 || it > 0) {
+          if (lane == 0) bulk_wait_read0();  // the previous store has read the staging tile
+          __syncwarp();
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 x;
+          x.x = pack_bf16x2(__uint_as_float(ov[p][8 * k + 0]), __uint_as_float(ov[p][8 * k + 1]));
+          x.y = pack_bf16x2(__uint_as_float(ov[p][8 * k + 2]), __uint_as_float(ov[p][8 * k + 3]));
+          x.z = pack_bf16x2(__uint_as_float(ov[p][8 * k + 4]), __uint_as_float(ov[p][8 * k + 5]));
+          x.w = pack_bf16x2(__uint_as_float(ov[p][8 * k + 6]), __uint_as_float(ov[p][8 * k + 7]));
+          *reinterpret_cast<uint4*>(stg + sw64_offset(lane, k)) = x;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && orow0 < T) {
+          tma_store_2d(&tmO, stg, h * D + ch * (D / 2) + p * 32, orow0);
+          bulk_commit();
+        }
+      }
     }
+    if (lane == 0) bulk_wait0();
   }
 
   tc_fence_before();

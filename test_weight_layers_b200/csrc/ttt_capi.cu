@@ -209,7 +209,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D bf16 tensor [outer][inner] with row stride `row_bytes`, 128-byte swizzled boxes.
 bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                uint32_t box_inner, uint32_t box_outer,
-               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -217,7 +218,7 @@ bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   return fn(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -456,9 +457,13 @@ int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t
   if (dt == TTT_BF16) {
     const int pair_tiles = (int)((T + 2 * TC_TILE - 1) / (2 * TC_TILE));
     const int n_items = pair_tiles * d.heads;
-    CUtensorMap tQ, tW, tW2;
+    CUtensorMap tQ, tW, tW2, tO;
     const uint64_t hd = (uint64_t)d.heads * d.d;
     if (!tmap_bf16(&tQ, Q, hd, (uint64_t)T, (uint64_t)ldq * 2, 64, TC_TILE)) return TTT_ERR_CUDA;
+    // output: [32 tokens x 32 columns] store boxes from 64-byte-swizzled staging tiles
+    if (!tmap_bf16(&tO, O, hd, (uint64_t)T, (uint64_t)ldo * 2, 32, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+      return TTT_ERR_CUDA;
     if (!tmap_bf16(&tW, w.wsh, (uint64_t)d.d, 3ull * d.heads * d.m, (uint64_t)d.d * 2, 64, 64)) return TTT_ERR_CUDA;
     if (!tmap_bf16(&tW2, w.w2b, (uint64_t)d.m, (uint64_t)d.heads * d.d, (uint64_t)d.m * 2, 64, (uint32_t)d.d / 2))
       return TTT_ERR_CUDA;
@@ -475,18 +480,17 @@ int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     ProfScope ps(TTT_PROF_APPLY, s);
-    __nv_bfloat16* Ob = (__nv_bfloat16*)O;
     const unsigned long long to = wait_timeout_ns();
     if (d.d == 192) {
       auto k = k_apply_tc<192>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<192>::ALLOC));
       cfg.dynamicSmemBytes = ApLayout<192>::ALLOC;
-      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, rq, Ob, ldo, T, d.heads, d.m, n_items, w.status, to));
+      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, tO, rq, T, d.heads, d.m, n_items, w.status, to));
     } else {
       auto k = k_apply_tc<128>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<128>::ALLOC));
       cfg.dynamicSmemBytes = ApLayout<128>::ALLOC;
-      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, rq, Ob, ldo, T, d.heads, d.m, n_items, w.status, to));
+      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, tO, rq, T, d.heads, d.m, n_items, w.status, to));
     }
     TTT_LAUNCHED();
   } else {
