@@ -19,9 +19,10 @@
 //
 // Roles (both kernels): warp 0 issues TMA loads, warp 1 issues MMAs (one
 // thread), warps 2..9 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
-// If the L2 normalisation of Q/K is on, the per-token inverse norm r_t scales
-// the epilogue: H1, H3 rows by r_t and dH1, dH3 rows by r_t (the GEMMs use the
-// raw keys/queries, which is exact because the norm is a row scale).
+// The gradient kernel reads K^ already normalised (fp16 copy written by the
+// preparation kernel).  In the apply kernel, if the L2 normalisation of Q is on,
+// the per-token inverse norm r_t scales the H1, H3 rows in the epilogue (the
+// GEMM uses the raw queries, which is exact because the norm is a row scale).
 #pragma once
 
 #include "common.cuh"
@@ -84,7 +85,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
     k_update_grad_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
                      const __grid_constant__ CUtensorMap tmW, const float* __restrict__ eta,
-                     const float* __restrict__ rk, float* __restrict__ partial, int64_t T, int H, int m,
+                     float* __restrict__ partial, int64_t T, int H, int m,
                      int tiles_total, int S, unsigned int* status, unsigned long long timeout_ns) {
   using L = UpdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -299,11 +300,7 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const int64_t t = (int64_t)(t_begin + i) * TC_TILE + row;
-      float e = 0.f, r = 0.f;
-      if (t < T) {
-        e = eta[t * H + h];
-        r = rk ? rk[t * H + h] : 1.f;
-      }
+      const float e = (t < T) ? eta[t * H + h] : 0.f;
       if (!__all_sync(0xffffffffu, mbar_wait(fdone, i & 1, g))) { ok = false; break; }
       tc_fence_after();
       uint32_t a1[32], a3[32], az[32];
@@ -316,29 +313,27 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_n(ffree, 32);  // F may now be overwritten by the next tile's forward
-      const float2 r2 = make_float2(r, r);
       // dH and U~ are stored as fp16 scaled by 2^8 (clear of fp16 subnormals); the
       // gradient readout multiplies by 2^-8, which is exact
-      const float2 er2 = make_float2(-e * r * GRAD_SCALE, -e * r * GRAD_SCALE);   // -eta * r
-      const float2 ne2 = make_float2(-e * GRAD_SCALE, -e * GRAD_SCALE);
+      const float2 ne2 = make_float2(-e * GRAD_SCALE, -e * GRAD_SCALE);  // -eta (scaled)
       const float2 half2 = make_float2(0.5f, 0.5f);
-      const float2 one2 = make_float2(1.f, 1.f);
+      const float2 mhalf2 = make_float2(-0.5f, -0.5f);
       uint32_t p1[16], p3[16], pu[16];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
-        const float2 h1 = __fmul2_rn(make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1])), r2);
-        const float2 h3 = __fmul2_rn(make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1])), r2);
+        const float2 h1 = make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1]));
+        const float2 h3 = make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1]));
         const float2 z = make_float2(__uint_as_float(az[j]), __uint_as_float(az[j + 1]));
         const float2 hh = __fmul2_rn(h1, half2);
         const float2 th = make_float2(tanh_approx(hh.x), tanh_approx(hh.y));
         const float2 s = __ffma2_rn(th, half2, half2);           // sigmoid(h1)
+        const float2 oms = __ffma2_rn(th, mhalf2, half2);        // 1 - sigmoid(h1)
         const float2 a = __fmul2_rn(h1, s);                      // SiLU(h1)
         const float2 u = __fmul2_rn(a, h3);
-        const float2 dz = __fmul2_rn(er2, z);                    // dL/du chained to the raw key
-        const float2 oms = __fadd2_rn(one2, make_float2(-s.x, -s.y));
+        const float2 dz = __fmul2_rn(ne2, z);                    // dL/du = -eta z
         const float2 qd = __ffma2_rn(a, oms, s);                 // SiLU'(h1) = s + a (1 - s)
-        const float2 d1 = __fmul2_rn(__fmul2_rn(dz, h3), qd);    // dL/dh1 (raw key)
-        const float2 d3 = __fmul2_rn(dz, a);                     // dL/dh3 (raw key)
+        const float2 d1 = __fmul2_rn(__fmul2_rn(dz, h3), qd);    // dL/dh1
+        const float2 d3 = __fmul2_rn(dz, a);                     // dL/dh3
         const float2 ut = __fmul2_rn(ne2, u);                    // -eta u
         p1[j >> 1] = pack_f16x2(d1.x, d1.y);
         p3[j >> 1] = pack_f16x2(d3.x, d3.y);

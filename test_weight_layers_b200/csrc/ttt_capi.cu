@@ -374,12 +374,12 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
     if (d.d == 192) {
       auto k = k_update_grad_tc<192>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<192>::ALLOC));
-      k<<<grid, UPD_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, rk, w.partial, T, d.heads, d.m,
+      k<<<grid, UPD_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, w.partial, T, d.heads, d.m,
                                                           tiles, S, w.status, wait_timeout_ns());
     } else {
       auto k = k_update_grad_tc<128>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<128>::ALLOC));
-      k<<<grid, UPD_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, rk, w.partial, T, d.heads, d.m,
+      k<<<grid, UPD_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, w.partial, T, d.heads, d.m,
                                                           tiles, S, w.status, wait_timeout_ns());
     }
     TTT_LAUNCHED();
