@@ -456,7 +456,7 @@ template <int D>
 __global__ void __launch_bounds__(AP_THREADS, 1)
     k_apply_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmW,
                const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmO,
-               const float* __restrict__ rq, int64_t T, int H, int m, int n_items, unsigned int* status,
+               int qnorm, int64_t T, int H, int m, int n_items, unsigned int* status,
                unsigned long long timeout_ns) {
   using L = ApLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* qfull = bars + 0;              // leader: TMA bytes of both CTAs
-  uint64_t* qfree = bars + 1;              // both: MMA done reading Q
+  uint64_t* qfree = bars + 1;              // both: MMA done reading Q (1) + this CTA's epilogue read its norms (256)
   uint64_t* w13full = bars + 2;            // [NS13] leader
   uint64_t* w13free = w13full + L::NS13;   // [NS13] both
   uint64_t* w2full = w13free + L::NS13;    // [NS2] leader
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
-    mbar_init(qfree, 1);
+    mbar_init(qfree, 1 + 256);
     for (int i = 0; i < L::NS13; ++i) {
       mbar_init(w13full + i, 1);
       mbar_init(w13free + i, 1);
@@ -640,11 +640,36 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     for (int item = pair; ok && item < n_items; item += npairs, ++it) {
       const int tile = item / H, h = item % H;
       const int64_t t = (int64_t)tile * 2 * TC_TILE + (int64_t)rank * TC_TILE + row;
-      const float r = (t < T) ? (rq ? rq[t * H + h] : 1.f) : 0.f;
+      float r = 1.f;
       for (int c = 0; c < nc; ++c, ++gc) {
         const int hb = gc & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(hfull + hb, (gc >> 1) & 1, g))) { ok = false; break; }
         tc_fence_after();
+        if (c == 0) {
+          // The first H of the item has read the query tile, so it is in shared
+          // memory; it stays there until this CTA's epilogue releases it (qfree).
+          // q^ = q / max(||q||, 1e-12): the GEMM used the raw query, so the
+          // inverse norm scales H1 and H3 rows here (rows past T were zero-filled).
+          if (qnorm) {
+            float ss = 0.f;
+#pragma unroll
+            for (int kb = 0; kb < L::KB; ++kb) {
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                const uint4 v = *reinterpret_cast<const uint4*>(smem + L::Q_OFF + kb * TC_BLK + sw128_offset(row, cc));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k2 = 0; k2 < 4; ++k2) {
+                  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[k2]));
+                  ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                }
+              }
+            }
+            r = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_n(qfree, 32);
+        }
         uint32_t a1[32], a3[32];
         tmem_ld32(tmem + lane_base + L::H_COL + hb * 128 + ch * 32, a1);
         tmem_ld32(tmem + lane_base + L::H_COL + hb * 128 + 64 + ch * 32, a3);

@@ -451,8 +451,11 @@ int run_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const t
   return TTT_OK;
 }
 
-int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t ldo, const float* rq, int64_t T,
-              const ttt_dims& d, ttt_dtype dt, const Ws& w, cudaStream_t s) {
+// Apply to T tokens.  qnorm: L2-normalise the queries per head (the tensor-core
+// kernel computes the norms from its query tile; the fp32 path writes them to
+// rq_buf [T][H] first).
+int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t ldo, int qnorm, float* rq_buf,
+              int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, cudaStream_t s) {
   if (T == 0) return TTT_OK;
   if (dt == TTT_BF16) {
     const int pair_tiles = (int)((T + 2 * TC_TILE - 1) / (2 * TC_TILE));
@@ -485,15 +488,20 @@ int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t
       auto k = k_apply_tc<192>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<192>::ALLOC));
       cfg.dynamicSmemBytes = ApLayout<192>::ALLOC;
-      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, tO, rq, T, d.heads, d.m, n_items, w.status, to));
+      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, tO, qnorm, T, d.heads, d.m, n_items, w.status, to));
     } else {
       auto k = k_apply_tc<128>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, ApLayout<128>::ALLOC));
       cfg.dynamicSmemBytes = ApLayout<128>::ALLOC;
-      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, tO, rq, T, d.heads, d.m, n_items, w.status, to));
+      TTT_CHECK(cudaLaunchKernelEx(&cfg, k, tQ, tW, tW2, tO, qnorm, T, d.heads, d.m, n_items, w.status, to));
     }
     TTT_LAUNCHED();
   } else {
+    const float* rq = nullptr;
+    if (qnorm) {
+      TTT_TRY(launch_rownorm_any(Q, ldq, T, d, dt, rq_buf, s));
+      rq = rq_buf;
+    }
     const size_t smem = (size_t)(F32_TT * d.d + 2 * F32_MS * d.d + d.d * F32_MS + F32_TT * F32_MS + F32_TT) * 4;
     TTT_CHECK(cudaFuncSetAttribute(k_apply_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     ProfScope ps(TTT_PROF_APPLY, s);
@@ -661,13 +669,8 @@ int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims, c
   if (T == 0) return TTT_OK;
   cudaStream_t s = (cudaStream_t)stream;
   Ws w = carve(ws, dims, T, dtype);
-  const float* rq = nullptr;
-  if (io->qk_l2norm) {
-    TTT_TRY(launch_rownorm_any(Q, ldq, T, dims, dtype, w.rq, s));
-    rq = w.rq;
-  }
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
-  return run_apply(W, Q, ldq, O, ldo, rq, T, dims, dtype, w, s);
+  return run_apply(W, Q, ldq, O, ldo, io->qk_l2norm, w.rq, T, dims, dtype, w, s);
 }
 
 int ttt_apply_noalloc(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims, const ttt_io_cfg* io,
@@ -705,12 +708,7 @@ int ttt_apply_noalloc(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims
     const int64_t tc = std::min(chunk, T - c0);
     const uint8_t* q = static_cast<const uint8_t*>(Q) + c0 * ldq * es;
     uint8_t* o = static_cast<uint8_t*>(O) + c0 * ldo * es;
-    const float* rq = nullptr;
-    if (io->qk_l2norm) {
-      TTT_TRY(launch_rownorm_any(q, ldq, tc, dims, dtype, rq_buf, s));
-      rq = rq_buf;
-    }
-    TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
+    TTT_TRY(run_apply(W, q, ldq, o, ldo, io->qk_l2norm, rq_buf, tc, dims, dtype, w, s));
   }
   return TTT_OK;
 }
@@ -743,19 +741,14 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
     const uint8_t* v = static_cast<const uint8_t*>(V) + c0 * ldv * es;
     uint8_t* o = static_cast<uint8_t*>(O) + c0 * ldo * es;
     const float* e = eta + c0 * dims.heads;
-    const float* rq = nullptr;
-    if (io->qk_l2norm) {
-      TTT_TRY(launch_rownorm_any(q, ldq, tc, dims, dtype, w.rq, s));
-      rq = w.rq;
-    }
     UpdOperands op;
     TTT_TRY(prepare_update_operands(k, ldk, v, ldv, tc, dims, dtype, io->qk_l2norm, w, s, &op));
-    if (order == 0) TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
+    if (order == 0) TTT_TRY(run_apply(W, q, ldq, o, ldo, io->qk_l2norm, w.rq, tc, dims, dtype, w, s));
     for (int st = 0; st < steps; ++st) {
       TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, e, op.rk, tc, dims, dtype, w, w.G, s));
       TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
     }
-    if (order == 1) TTT_TRY(run_apply(W, q, ldq, o, ldo, rq, tc, dims, dtype, w, s));
+    if (order == 1) TTT_TRY(run_apply(W, q, ldq, o, ldo, io->qk_l2norm, w.rq, tc, dims, dtype, w, s));
   }
   return TTT_OK;
 }
