@@ -167,6 +167,39 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
                 int64_t T, int64_t chunk, int order, int steps, const ttt_ns_cfg* ns, ttt_dims dims,
                 const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
+/* The whole layer over HOST-resident tokens, with the host<->device copies
+ * overlapped with the computation (no counterpart in the pages: this is how a
+ * caller whose tokens live in host memory runs the layer without paying for
+ * the copies and the computation one after the other).
+ *  - hQ, hK, hV, hO: HOST pointers to dense [T][H*d] token matrices (dtype as
+ *    given), hEta: HOST float [T][H].  They should be page-locked (pinned)
+ *    memory; pageable memory works, but its copies do not overlap.
+ *  - dbuf: DEVICE staging area of ttt_host_buffer_bytes(dims, T, dtype, conv)
+ *    bytes, 256-byte aligned, owned by the caller; it receives the device
+ *    copies of Q, K, V, eta and O (and V after ShortConv2D when conv = 1).
+ *  - ws: the usual workspace, for T tokens (chunk = 0) or `chunk` tokens.
+ *  - chunk = 0: `steps` Muon steps over all T tokens (as ttt_update), then the
+ *    apply to all T queries.  K, V, eta arrive in token blocks; the first
+ *    step's gradient is computed block by block while later blocks are still
+ *    being copied (block gradients are summed, so the result equals ttt_update
+ *    up to the order of that sum), and each block of O is copied back as soon
+ *    as it has been computed, while later queries are still arriving.
+ *  - chunk > 0: the causal carry of ttt_chunked with order 0; chunk c+1 is
+ *    copied in while chunk c is computed and O of chunk c is copied back
+ *    meanwhile.
+ *  - taps (device float [H*d][3][3]) non-null applies ShortConv2D to V over
+ *    frames of grid_h x grid_w tokens first (T must be whole frames); the
+ *    token blocks of chunk = 0 are then whole frames, and chunk must be too.
+ *  - io: only qk_l2norm is read (host rows are dense).
+ * On return the work is queued on `stream`: when `stream` has completed, hO
+ * holds the outputs and W the updated weights.  The library creates two copy
+ * streams and a pool of events per device on first use and keeps them. */
+size_t ttt_host_buffer_bytes(ttt_dims dims, int64_t T, ttt_dtype dtype, int conv);
+int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV, const float* hEta, void* hO,
+                   int64_t T, int64_t chunk, int steps, const ttt_ns_cfg* ns, const float* taps, int grid_h,
+                   int grid_w, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, void* dbuf, size_t dbuf_bytes,
+                   void* ws, size_t ws_bytes, void* stream);
+
 /* Diagnostic for the timeout path: launches one single-warp kernel that waits on
  * a barrier nothing ever signals, with a wait limit of `timeout_us`
  * microseconds.  The wait gives up, records TTT_ERR_TIMEOUT in the workspace

@@ -388,13 +388,18 @@ __global__ void k_shadow(const float* __restrict__ W1, const float* __restrict__
 // ---------------------------------------------------------------------------
 // Deterministic split-K reduction: G[i] = sum_{s=0..S-1} P[s][i] in that order.
 
-__global__ void k_reduce_splits(const float* __restrict__ P, int S, int64_t n, float* __restrict__ G) {
+// G = sum over the S split partials (accumulate = 1: G += that sum), fixed order.
+__global__ void k_reduce_splits(const float* __restrict__ P, int S, int64_t n, float* __restrict__ G, int accumulate) {
   const int64_t n4 = n / 4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
     float4 acc = reinterpret_cast<const float4*>(P)[i];
     for (int s = 1; s < S; ++s) {
       float4 v = reinterpret_cast<const float4*>(P + (int64_t)s * n)[i];
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    if (accumulate) {
+      const float4 g = reinterpret_cast<const float4*>(G)[i];
+      acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
     }
     reinterpret_cast<float4*>(G)[i] = acc;
   }

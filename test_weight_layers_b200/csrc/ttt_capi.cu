@@ -348,11 +348,13 @@ int prepare_update_operands(const void* K, int64_t ldk, const void* V, int64_t l
 
 // gradient over T tokens -> G (fp32, [3][H*m*d]); shadow of W must be current.
 // bf16 mode: K, V are the fp16 operands written by launch_prep_kv (ld = H*d, K^ normalised).
+// accumulate = true adds the gradient to G instead of overwriting it.
 int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta,
-             const float* rk, int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, float* G, cudaStream_t s) {
+             const float* rk, int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, float* G, cudaStream_t s,
+             bool accumulate = false) {
   const int64_t n = (int64_t)d.heads * d.m * d.d;
   if (T == 0) {
-    TTT_CHECK(cudaMemsetAsync(G, 0, 3 * n * sizeof(float), s));
+    if (!accumulate) TTT_CHECK(cudaMemsetAsync(G, 0, 3 * n * sizeof(float), s));
     return TTT_OK;
   }
   int S = 1;
@@ -396,7 +398,7 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
     TTT_LAUNCHED();
   }
   ProfScope ps(TTT_PROF_REDUCE, s);
-  k_reduce_splits<<<grid1d(3 * n / 4, 256), 256, 0, s>>>(w.partial, S, 3 * n, G);
+  k_reduce_splits<<<grid1d(3 * n / 4, 256), 256, 0, s>>>(w.partial, S, 3 * n, G, accumulate ? 1 : 0);
   TTT_LAUNCHED();
   return TTT_OK;
 }
@@ -540,6 +542,66 @@ int noalloc_scratch(void** out) {
     g_noalloc_addr[dev] = p;
   }
   *out = g_noalloc_addr[dev];
+  return TTT_OK;
+}
+
+// ---- host-buffer layer (ttt_layer_host): two copy streams and a pool of
+// events per device, created on first use and kept for the process lifetime
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+std::mutex g_pipe_mu;  // held while a call queues its work (the events are shared)
+HostPipe g_pipes[64];
+constexpr int kHostBlocks = 16;  // token blocks of the bidirectional host pipeline
+
+int host_pipe(HostPipe** out, size_t n_events) {
+  int dev = 0;
+  TTT_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return TTT_ERR_CUDA;
+  HostPipe& p = g_pipes[dev];
+  if (!p.h2d) TTT_CHECK(cudaStreamCreateWithFlags(&p.h2d, cudaStreamNonBlocking));
+  if (!p.d2h) TTT_CHECK(cudaStreamCreateWithFlags(&p.d2h, cudaStreamNonBlocking));
+  while (p.ev.size() < n_events) {
+    cudaEvent_t e;
+    TTT_CHECK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    p.ev.push_back(e);
+  }
+  *out = &p;
+  return TTT_OK;
+}
+
+// dbuf layout: Q, K, V, O [T][H*d], eta [T][H], then V after ShortConv2D (conv)
+struct HostLayout {
+  size_t q, k, v, o, eta, vc, total;
+};
+HostLayout host_layout(const ttt_dims& d, int64_t T, ttt_dtype dt, bool conv) {
+  const size_t tm = up256((size_t)std::max<int64_t>(T, 1) * d.heads * d.d * esize(dt));
+  HostLayout L{};
+  L.q = 0;
+  L.k = tm;
+  L.v = 2 * tm;
+  L.o = 3 * tm;
+  L.eta = 4 * tm;
+  L.vc = L.eta + up256((size_t)std::max<int64_t>(T, 1) * d.heads * 4);
+  L.total = L.vc + (conv ? tm : 0);
+  return L;
+}
+
+int launch_conv(const void* V, void* Vout, const float* taps, int64_t frames, int gh, int gw, int C, ttt_dtype dt,
+                cudaStream_t s) {
+  if (frames == 0) return TTT_OK;
+  const int vn = dt == TTT_BF16 ? 8 : 4;
+  const int gv = CONV_GROUP / vn;
+  const dim3 block(gv, 256 / gv);
+  const dim3 grid((unsigned)frames, (C + CONV_GROUP - 1) / CONV_GROUP);
+  ProfScope ps(TTT_PROF_CONV, s);
+  if (dt == TTT_BF16)
+    k_shortconv<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)V, C, (__nv_bfloat16*)Vout, C, taps,
+                                                      (int)frames, gh, gw, C, 0);
+  else
+    k_shortconv<float><<<grid, block, 0, s>>>((const float*)V, C, (float*)Vout, C, taps, (int)frames, gh, gw, C, 0);
+  TTT_LAUNCHED();
   return TTT_OK;
 }
 
@@ -750,6 +812,169 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
     }
     if (order == 1) TTT_TRY(run_apply(W, q, ldq, o, ldo, io->qk_l2norm, w.rq, tc, dims, dtype, w, s));
   }
+  return TTT_OK;
+}
+
+size_t ttt_host_buffer_bytes(ttt_dims dims, int64_t T, ttt_dtype dtype, int conv) {
+  if (!dims_ok(dims) || T < 0 || (dtype != TTT_FP32 && dtype != TTT_BF16)) return 0;
+  return host_layout(dims, T, dtype, conv != 0).total;
+}
+
+int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV, const float* hEta, void* hO,
+                   int64_t T, int64_t chunk, int steps, const ttt_ns_cfg* ns, const float* taps, int grid_h,
+                   int grid_w, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, void* dbuf, size_t dbuf_bytes,
+                   void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || chunk < 0 || steps < 0) return TTT_ERR_INVALID;
+  const int64_t wsT = chunk > 0 ? std::min<int64_t>(chunk, T) : T;
+  TTT_TRY(check_common(dims, dtype, wsT, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  if (steps > 0) TTT_TRY(check_ns(ns));
+  if (!io) io = &kDefaultIo;
+  if (T == 0) return TTT_OK;
+  if (!hQ || !hK || !hV || !hEta || !hO || !dbuf) return TTT_ERR_INVALID;
+  const bool conv = taps != nullptr;
+  const int64_t hd = (int64_t)dims.heads * dims.d;
+  const int64_t fr = conv ? (int64_t)grid_h * grid_w : 1;
+  if (conv) {
+    if (grid_h < 1 || grid_w < 1 || T % fr || (chunk > 0 && chunk % fr)) return TTT_ERR_INVALID;
+    if (hd % 8) return TTT_ERR_UNSUPPORTED;
+  }
+  const HostLayout L = host_layout(dims, T, dtype, conv);
+  if (dbuf_bytes < L.total) return TTT_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(dbuf) & 255u) return TTT_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t es = esize(dtype);
+  const size_t row = (size_t)hd * es;
+  uint8_t* base = static_cast<uint8_t*>(dbuf);
+  uint8_t* dQ = base + L.q;
+  uint8_t* dK = base + L.k;
+  uint8_t* dV = base + L.v;
+  uint8_t* dO = base + L.o;
+  uint8_t* dVc = base + L.vc;
+  float* dEta = reinterpret_cast<float*>(base + L.eta);
+  const uint8_t* cQ = static_cast<const uint8_t*>(hQ);
+  const uint8_t* cK = static_cast<const uint8_t*>(hK);
+  const uint8_t* cV = static_cast<const uint8_t*>(hV);
+  uint8_t* cO = static_cast<uint8_t*>(hO);
+  // token blocks: the chunks (chunk > 0), else kHostBlocks blocks of whole tiles (or frames)
+  int64_t bt = chunk;
+  if (chunk == 0) {
+    const int64_t unit = conv ? fr : TC_TILE;
+    const int64_t units = (T + unit - 1) / unit;
+    bt = ((units + kHostBlocks - 1) / kHostBlocks) * unit;
+  }
+  const int64_t nb = (T + bt - 1) / bt;
+  std::lock_guard<std::mutex> lk(g_pipe_mu);
+  HostPipe* P = nullptr;
+  TTT_TRY(host_pipe(&P, (size_t)(3 * nb + 3)));
+  cudaEvent_t* ev = P->ev.data();
+  cudaEvent_t ev_start = ev[0], ev_h2d_end = ev[1], ev_d2h_end = ev[2];
+  cudaEvent_t* ev_in = ev + 3;            // [nb] K, V, eta (and Q in chunk mode) of block b on the device
+  cudaEvent_t* ev_q = ev + 3 + nb;        // [nb] Q of block b on the device (chunk = 0)
+  cudaEvent_t* ev_o = ev + 3 + 2 * nb;    // [nb] O of block b computed
+  // the copies must not overwrite dbuf while earlier work on `stream` still uses it
+  TTT_CHECK(cudaEventRecord(ev_start, s));
+  TTT_CHECK(cudaStreamWaitEvent(P->h2d, ev_start, 0));
+  TTT_CHECK(cudaStreamWaitEvent(P->d2h, ev_start, 0));
+  auto up = [&](uint8_t* dst, const uint8_t* src, size_t bytes) {
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, P->h2d);
+  };
+  auto body = [&]() -> int {
+    for (int64_t b = 0; b < nb; ++b) {
+      const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
+      TTT_CHECK(up(dK + t0 * row, cK + t0 * row, tb * row));
+      TTT_CHECK(up(dV + t0 * row, cV + t0 * row, tb * row));
+      TTT_CHECK(up(reinterpret_cast<uint8_t*>(dEta + t0 * dims.heads),
+                   reinterpret_cast<const uint8_t*>(hEta + t0 * dims.heads), (size_t)tb * dims.heads * 4));
+      if (chunk > 0) TTT_CHECK(up(dQ + t0 * row, cQ + t0 * row, tb * row));
+      TTT_CHECK(cudaEventRecord(ev_in[b], P->h2d));
+    }
+    if (chunk == 0)
+      for (int64_t b = 0; b < nb; ++b) {
+        const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
+        TTT_CHECK(up(dQ + t0 * row, cQ + t0 * row, tb * row));
+        TTT_CHECK(cudaEventRecord(ev_q[b], P->h2d));
+      }
+    Ws w = carve(ws, dims, wsT, dtype);
+    if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
+    // V of block b after the optional ShortConv2D
+    auto vsrc = [&](int64_t t0, int64_t tb) -> const uint8_t* {
+      if (!conv) return dV + t0 * row;
+      if (launch_conv(dV + t0 * row, dVc + t0 * row, taps, tb / fr, grid_h, grid_w, (int)hd, dtype, s) != TTT_OK)
+        return nullptr;
+      return dVc + t0 * row;
+    };
+    auto apply_block = [&](int64_t b, float* rq_buf) -> int {
+      const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
+      TTT_TRY(run_apply(W, dQ + t0 * row, hd, dO + t0 * row, hd, io->qk_l2norm, rq_buf, tb, dims, dtype, w, s));
+      TTT_CHECK(cudaEventRecord(ev_o[b], s));
+      TTT_CHECK(cudaStreamWaitEvent(P->d2h, ev_o[b], 0));
+      TTT_CHECK(cudaMemcpyAsync(cO + t0 * row, dO + t0 * row, tb * row, cudaMemcpyDeviceToHost, P->d2h));
+      return TTT_OK;
+    };
+    if (chunk > 0) {
+      // causal carry, order 0: O_c = f_(W_(c-1))(Q_c), then the update on chunk c
+      for (int64_t b = 0; b < nb; ++b) {
+        const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
+        TTT_CHECK(cudaStreamWaitEvent(s, ev_in[b], 0));
+        TTT_TRY(apply_block(b, w.rq));
+        if (steps == 0) continue;
+        const uint8_t* v = vsrc(t0, tb);
+        if (!v) return TTT_ERR_CUDA;
+        UpdOperands op;
+        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, tb, dims, dtype, io->qk_l2norm, w, s, &op));
+        for (int st = 0; st < steps; ++st) {
+          TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s));
+          TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+        }
+      }
+      return TTT_OK;
+    }
+    if (steps > 0) {
+      // first step: preparation and gradient block by block as the blocks land
+      for (int64_t b = 0; b < nb; ++b) {
+        const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
+        TTT_CHECK(cudaStreamWaitEvent(s, ev_in[b], 0));
+        const uint8_t* v = vsrc(t0, tb);
+        if (!v) return TTT_ERR_CUDA;
+        Ws wb = w;  // per-token operand buffers shifted to the block
+        if (dtype == TTT_BF16) {
+          wb.kh16 = w.kh16 + t0 * hd;
+          wb.vh16 = w.vh16 + t0 * hd;
+        } else {
+          wb.rk = w.rk + t0 * dims.heads;
+        }
+        UpdOperands op;
+        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, tb, dims, dtype, io->qk_l2norm, wb, s, &op));
+        TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s,
+                         b > 0));
+      }
+      TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+      // further steps re-read the prepared operands of all T tokens
+      UpdOperands full;
+      if (dtype == TTT_BF16)
+        full = {w.kh16, hd, w.vh16, hd, nullptr};
+      else
+        full = {dK, hd, conv ? dVc : dV, hd, io->qk_l2norm ? w.rk : nullptr};
+      for (int st = 1; st < steps; ++st) {
+        TTT_TRY(run_grad(W, full.K, full.ldk, full.V, full.ldv, dEta, full.rk, T, dims, dtype, w, w.G, s));
+        TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+      }
+    }
+    for (int64_t b = 0; b < nb; ++b) {
+      TTT_CHECK(cudaStreamWaitEvent(s, ev_q[b], 0));
+      TTT_TRY(apply_block(b, w.rq + b * bt * dims.heads));
+    }
+    return TTT_OK;
+  };
+  const int rc = body();
+  // `stream` completes only after both copy streams (also when queueing failed midway)
+  const cudaError_t e1 = cudaEventRecord(ev_h2d_end, P->h2d);
+  const cudaError_t e2 = cudaEventRecord(ev_d2h_end, P->d2h);
+  const cudaError_t e3 = cudaStreamWaitEvent(s, ev_h2d_end, 0);
+  const cudaError_t e4 = cudaStreamWaitEvent(s, ev_d2h_end, 0);
+  if (rc != TTT_OK) return rc;
+  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess || e4 != cudaSuccess) return TTT_ERR_CUDA;
   return TTT_OK;
 }
 

@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
             "ttt_apply_noalloc": (I, [Weights, P, P, I64, Dims, ctypes.POINTER(IOCfg), I, P]),
             "ttt_chunked": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), Dims,
                                 ctypes.POINTER(IOCfg), I, P, SZ, P]),
+            "ttt_host_buffer_bytes": (SZ, [Dims, I64, I, I]),
+            "ttt_layer_host": (I, [Weights, P, P, P, P, P, I64, I64, I, ctypes.POINTER(NSCfg), P, I, I, Dims,
+                                   ctypes.POINTER(IOCfg), I, P, SZ, P, SZ, P]),
             "ttt_status_string": (ctypes.c_char_p, [I]),
             "ttt_selftest_wait_timeout": (I, [P, SZ, ctypes.c_uint, P]),
             "ttt_launch_count": (ctypes.c_uint64, []),
@@ -186,6 +189,27 @@ def ttt_chunked(W: Weights, Q, K, V, eta, O, T, chunk, order, steps, ns: NSCfg, 
     _check("ttt_chunked", lib().ttt_chunked(W, _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(O), T, chunk, order, steps,
                                             ctypes.byref(ns), dm, ctypes.byref(io), dtype_code(Q.dtype), _ptr(ws),
                                             ws.numel(), _stream(stream)))
+
+
+def ttt_host_buffer_bytes(dm: Dims, T: int, dtype: int, conv: bool = False) -> int:
+    return int(lib().ttt_host_buffer_bytes(dm, T, dtype, 1 if conv else 0))
+
+
+def host_buffer(dm: Dims, T: int, dtype: int, conv: bool = False, device="cuda") -> torch.Tensor:
+    """Device staging area for ttt_layer_host (256-byte aligned, as torch allocations are)."""
+    n = ttt_host_buffer_bytes(dm, T, dtype, conv)
+    if n == 0:
+        raise TTTError("ttt_host_buffer_bytes", TTT_ERR_INVALID, "invalid dims")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def ttt_layer_host(W: Weights, hQ, hK, hV, hEta, hO, T, chunk, steps, ns: NSCfg, dm: Dims, io: IOCfg, dbuf, ws,
+                   taps=None, grid_h=0, grid_w=0, stream=None):
+    """hQ, hK, hV, hEta, hO are host (pinned CPU) tensors; dbuf, ws, taps and W are on the device."""
+    _check("ttt_layer_host", lib().ttt_layer_host(
+        W, _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hEta), _ptr(hO), T, chunk, steps, ctypes.byref(ns), _ptr(taps), grid_h,
+        grid_w, dm, ctypes.byref(io), dtype_code(hQ.dtype), _ptr(dbuf), dbuf.numel(), _ptr(ws), ws.numel(),
+        _stream(stream)))
 
 
 def ttt_selftest_wait_timeout(ws, timeout_us: int, stream=None):
