@@ -505,79 +505,118 @@ __global__ void k_ns_finish(const float* __restrict__ X, float* __restrict__ D, 
   }
 }
 
-// Batched C = alpha * A * op(B) + beta * Cin, fp32, 64x64 tiles, 256 threads, 4x4 per thread.
-// A: [M][K] (lda), op(B) = B [K][N] (ldb) or, with TRANS_B, B^T with B [N][K].
-// Global loads of the next 16-deep K slice are issued before the current slice's FMAs.
-template <bool TRANS_B>
-__global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const float* __restrict__ A, int lda, int64_t sA,
-                                                  const float* __restrict__ B, int ldb, int64_t sB, float* __restrict__ C,
-                                                  int ldc, int64_t sC, const float* __restrict__ Cin, float alpha,
-                                                  float beta) {
-  __shared__ __align__(16) float As[2][16][64];
-  __shared__ __align__(16) float Bs[2][16][64];
-  const int b = blockIdx.z;
-  A += b * sA;
-  B += b * sB;
-  C += b * sC;
-  if (Cin) Cin += b * sC;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+// ---- fp32 64x64 tile products of the Newton-Schulz iteration (CUDA cores)
+
+constexpr int NSC_KMAX = 192;            // K extent staged in shared memory at once
+constexpr int NSC_SA = NSC_KMAX + 4;     // row stride of the staged A tile (floats)
+
+// dynamic shared memory: A tile [64][NSC_SA] then the B tile, [NSC_KMAX][64] or
+// (B = X^T) [64][NSC_SA]
+constexpr int NSC_B_FLOATS = 64 * NSC_SA > NSC_KMAX * 64 ? 64 * NSC_SA : NSC_KMAX * 64;
+constexpr int NSC_DYN_BYTES = (64 * NSC_SA + NSC_B_FLOATS) * 4;
+
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 fills zeros
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Tile column of acc[.][j] for thread column tx (see nsc_tile).
+__device__ __forceinline__ int nsc_col(int tx, int j, bool bt) { return bt ? tx + 16 * j : 4 * tx + j; }
+
+// acc += A(m0 + i, k0 + k) B(k0 + k, n0 + j) over k < K (K <= NSC_KMAX, K % 4 == 0)
+// for the 64x64 tile; thread (ty, tx) = (tid / 16, tid % 16) owns rows 4 ty ..
+// 4 ty + 3 and columns nsc_col(tx, 0..3, BT).  Both operands are staged whole in
+// shared memory by 16-byte asynchronous copies all in flight together (one L2
+// round trip per tile), then the FMAs run from shared memory.  A: rows of the
+// row-major matrix a (lda), rows >= Mv read as 0.  B (BT = false): rows k of
+// the row-major matrix bsrc (ldb), columns >= Nv read as 0; BT = true:
+// B(k, j) = bsrc[(n0 + j) ldb + k0 + k] (B = X^T), staged as rows j.
+// Leading dimensions and k0 are multiples of 4 floats.
+template <bool BT>
+__device__ __forceinline__ void nsc_tile(const float* __restrict__ a, int lda, int m0, int Mv,
+                                         const float* __restrict__ bsrc, int ldb, int n0, int Nv, int k0, int K,
+                                         float (&acc)[4][4], float* smA, float* smB) {
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  // loader mapping: 4 elements per thread per operand per slice
-  float ra[4], rb[4];
-  auto load = [&](int k0) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = tid + 256 * q;
-      {  // A slice [64 m][16 k]: i -> (mm = i / 16, kk = i % 16)
-        const int kk = i & 15, mm = i >> 4, gm = m0 + mm, gk = k0 + kk;
-        ra[q] = (gm < M && gk < K) ? A[(int64_t)gm * lda + gk] : 0.f;
-      }
-      if (TRANS_B) {
-        const int kk = i & 15, nn = i >> 4, gn = n0 + nn, gk = k0 + kk;
-        rb[q] = (gn < N && gk < K) ? B[(int64_t)gn * ldb + gk] : 0.f;
-      } else {
-        const int nn = i & 63, kk = i >> 6, gn = n0 + nn, gk = k0 + kk;
-        rb[q] = (gn < N && gk < K) ? B[(int64_t)gk * ldb + gn] : 0.f;
-      }
+  const int kq = K / 4;
+  __syncthreads();  // the previous tile's reads of smA / smB are done
+  for (int idx = tid; idx < 64 * kq; idx += 256) {
+    const int row = idx / kq, q = idx % kq;
+    const bool in = m0 + row < Mv;
+    cp_async16(smA + row * NSC_SA + 4 * q, a + (int64_t)(in ? m0 + row : 0) * lda + k0 + 4 * q, in ? 16u : 0u);
+  }
+  if (!BT) {
+    for (int idx = tid; idx < K * 16; idx += 256) {
+      const int k = idx >> 4, q = idx & 15;
+      const bool in = n0 + 4 * q < Nv;
+      cp_async16(smB + k * 64 + 4 * q, bsrc + (int64_t)(k0 + k) * ldb + (in ? n0 + 4 * q : 0), in ? 16u : 0u);
     }
-  };
-  auto stash = [&](int buf) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = tid + 256 * q;
-      As[buf][i & 15][i >> 4] = ra[q];
-      if (TRANS_B) Bs[buf][i & 15][i >> 4] = rb[q];
-      else Bs[buf][i >> 6][i & 63] = rb[q];
+  } else {
+    // B^T: rows n0 + j of bsrc, stored like A ([64][NSC_SA])
+    for (int idx = tid; idx < 64 * kq; idx += 256) {
+      const int row = idx / kq, q = idx % kq;
+      const bool in = n0 + row < Nv;
+      cp_async16(smB + row * NSC_SA + 4 * q, bsrc + (int64_t)(in ? n0 + row : 0) * ldb + k0 + 4 * q, in ? 16u : 0u);
     }
-  };
-  float acc[4][4] = {};
-  load(0);
-  stash(0);
+  }
+  cp_async_wait_all();
   __syncthreads();
-  int buf = 0;
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    const bool more = k0 + 16 < K;
-    if (more) load(k0 + 16);
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-      const float4 bv = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-      const float a4[4] = {av.x, av.y, av.z, av.w};
+  const float* ar = smA + (ty * 4) * NSC_SA;
+  if (!BT) {
+#pragma unroll 8
+    for (int k = 0; k < K; ++k) {
+      const float a4[4] = {ar[k], ar[NSC_SA + k], ar[2 * NSC_SA + k], ar[3 * NSC_SA + k]};
+      const float4 bv = *reinterpret_cast<const float4*>(smB + k * 64 + tx * 4);
       const float b4[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
     }
-    if (more) stash(buf ^ 1);
-    __syncthreads();
-    buf ^= 1;
+  } else {
+    // columns tx, tx + 16, tx + 32, tx + 48 (conflict-free reads of the row-stored B^T)
+    const float* br = smB + tx * NSC_SA;
+#pragma unroll 8
+    for (int k = 0; k < K; ++k) {
+      const float a4[4] = {ar[k], ar[NSC_SA + k], ar[2 * NSC_SA + k], ar[3 * NSC_SA + k]};
+      const float b4[4] = {br[k], br[16 * NSC_SA + k], br[32 * NSC_SA + k], br[48 * NSC_SA + k]};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+    }
   }
+}
+
+// Batched C = alpha * A * B + beta * Cin, fp32, one 64x64 output tile per CTA
+// (256 threads), K staged in shared memory in pieces of NSC_KMAX.  A [M][K]
+// (lda), B [K][N] (ldb); leading dimensions and K are multiples of 4.
+// Dynamic shared memory: NSC_DYN_BYTES.
+__global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const float* __restrict__ A, int lda,
+                                                  int64_t sA, const float* __restrict__ B, int ldb, int64_t sB,
+                                                  float* __restrict__ C, int ldc, int64_t sC,
+                                                  const float* __restrict__ Cin, float alpha, float beta) {
+  extern __shared__ __align__(16) float gemm_dyn[];
+  float* smA = gemm_dyn;
+  float* smB = gemm_dyn + 64 * NSC_SA;
+  const int b = blockIdx.z;
+  A += b * sA;
+  B += b * sB;
+  C += b * sC;
+  if (Cin) Cin += b * sC;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += NSC_KMAX)
+    nsc_tile<false>(A, lda, m0, M, B, ldb, n0, N, k0, min(NSC_KMAX, K - k0), acc, smA, smB);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
+      const int gm = m0 + ty * 4 + i, gn = n0 + nsc_col(tx, j, false);
       if (gm < M && gn < N) {
         float v = alpha * acc[i][j];
         if (Cin) v = fmaf(beta, Cin[(int64_t)gm * ldc + gn], v);
@@ -590,13 +629,14 @@ __global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const flo
 // 64x64 tiles only (A is symmetric), split-K over NS_GRAM_SPLIT slices of the
 // long dimension for parallelism.  grid (tiles, NS_GRAM_SPLIT, batch); partial
 // P[s][b][i][j] for the tile's (i, j); k_gram_reduce sums the slices in fixed
-// order and mirrors the lower triangle.
+// order and mirrors the lower triangle.  Dynamic shared memory: NSC_DYN_BYTES.
 constexpr int NS_GRAM_SPLIT = 4;
 
 __global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float* __restrict__ X, int64_t sX,
                                                       float* __restrict__ P) {
-  __shared__ __align__(16) float As[2][16][64];
-  __shared__ __align__(16) float Bs[2][16][64];
+  extern __shared__ __align__(16) float gram_dyn[];
+  float* smA = gram_dyn;
+  float* smB = gram_dyn + 64 * NSC_SA;
   const int rt = (r + 63) / 64;
   // tile index -> (ti <= tj) in row-major upper-triangular order
   int t = blockIdx.x, ti = 0;
@@ -607,55 +647,16 @@ __global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float*
   const int k_begin = s * kper, k_end = min(c, k_begin + kper);
   const float* x = X + (int64_t)b * sX;
   const int m0 = ti * 64, n0 = tj * 64;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  float ra[4], rb[4];
-  auto load = [&](int k0) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = tid + 256 * q, kk = i & 15, mm = i >> 4, gk = k0 + kk;
-      ra[q] = (m0 + mm < r && gk < k_end) ? x[(int64_t)(m0 + mm) * c + gk] : 0.f;
-      rb[q] = (n0 + mm < r && gk < k_end) ? x[(int64_t)(n0 + mm) * c + gk] : 0.f;
-    }
-  };
-  auto stash = [&](int buf) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = tid + 256 * q;
-      As[buf][i & 15][i >> 4] = ra[q];
-      Bs[buf][i & 15][i >> 4] = rb[q];
-    }
-  };
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float acc[4][4] = {};
-  int buf = 0;
-  if (k_begin < k_end) {
-    load(k_begin);
-    stash(0);
-  }
-  __syncthreads();
-  for (int k0 = k_begin; k0 < k_end; k0 += 16) {
-    const bool more = k0 + 16 < k_end;
-    if (more) load(k0 + 16);
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-      const float4 bv = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-      const float a4[4] = {av.x, av.y, av.z, av.w};
-      const float b4[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
-    }
-    if (more) stash(buf ^ 1);
-    __syncthreads();
-    buf ^= 1;
-  }
+  for (int k0 = k_begin; k0 < k_end; k0 += NSC_KMAX)
+    nsc_tile<true>(x, c, m0, r, x, c, n0, r, k0, min(NSC_KMAX, k_end - k0), acc, smA, smB);
   float* out = P + ((int64_t)s * gridDim.z + b) * (int64_t)r * r;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
+      const int gm = m0 + ty * 4 + i, gn = n0 + nsc_col(tx, j, true);
       if (gm < r && gn < r) out[(int64_t)gm * r + gn] = acc[i][j];
     }
 }

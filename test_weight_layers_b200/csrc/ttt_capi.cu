@@ -420,15 +420,17 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
     float* X = w.X;
     float* X2 = w.X2;
     const int rt = (r + 63) / 64, ct = (c + 63) / 64;
+    TTT_CHECK(cudaFuncSetAttribute(k_gram_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, NSC_DYN_BYTES));
+    TTT_CHECK(cudaFuncSetAttribute(k_gemm_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, NSC_DYN_BYTES));
     for (int it = 0; it < ns.iters; ++it) {
-      k_gram_partial<<<dim3(rt * (rt + 1) / 2, NS_GRAM_SPLIT, nb), 256, 0, s>>>(r, c, X, n, w.gram);
+      k_gram_partial<<<dim3(rt * (rt + 1) / 2, NS_GRAM_SPLIT, nb), 256, NSC_DYN_BYTES, s>>>(r, c, X, n, w.gram);
       TTT_LAUNCHED();
       k_gram_reduce<<<grid1d((int64_t)nb * r * r, 256), 256, 0, s>>>(r, nb, w.gram, w.A);
       TTT_LAUNCHED();
-      k_gemm_f32<false><<<dim3(rt, rt, nb), 256, 0, s>>>(r, r, r, w.A, r, (int64_t)r * r, w.A, r, (int64_t)r * r, w.B,
+      k_gemm_f32<<<dim3(rt, rt, nb), 256, NSC_DYN_BYTES, s>>>(r, r, r, w.A, r, (int64_t)r * r, w.A, r, (int64_t)r * r, w.B,
                                                           r, (int64_t)r * r, w.A, ns.c, ns.b);
       TTT_LAUNCHED();
-      k_gemm_f32<false><<<dim3(ct, rt, nb), 256, 0, s>>>(r, c, r, w.B, r, (int64_t)r * r, X, c, n, X2, c, n, X, 1.f,
+      k_gemm_f32<<<dim3(ct, rt, nb), 256, NSC_DYN_BYTES, s>>>(r, c, r, w.B, r, (int64_t)r * r, X, c, n, X2, c, n, X, 1.f,
                                                           ns.a);
       TTT_LAUNCHED();
       std::swap(X, X2);
