@@ -358,6 +358,107 @@ __global__ void __launch_bounds__(256, 4) k_shortconv(const T* __restrict__ V, i
   }
 }
 
+// Banded ShortConv2D: CTA = (64-channel group, frame slot); the frame is walked
+// in bands of BR output rows.  Each band's BR + 2 input rows (one halo row on
+// each side, zero-filled outside the frame) are staged in shared memory with
+// 16-byte asynchronous copies, double-buffered so the next band loads while
+// this one is computed; the 3x3 sums then read shared memory only.  Frames past
+// gridDim.y are taken in a grid-stride loop.  Dynamic shared memory:
+// conv_band_smem(BR, gw, sizeof(T)).
+__host__ __device__ constexpr size_t conv_band_bytes(int BR, int gw, int esz) {
+  return (size_t)(BR + 2) * gw * CONV_GROUP * esz;
+}
+__host__ __device__ constexpr size_t conv_band_smem(int BR, int gw, int esz) {
+  return 9 * CONV_GROUP * sizeof(float) + 2 * conv_band_bytes(BR, gw, esz);
+}
+
+__device__ __forceinline__ void cp_async16_cg(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256, 2) k_shortconv_band(const T* __restrict__ V, int64_t ldv, T* __restrict__ out,
+                                                        int64_t ldo, const float* __restrict__ taps, int N, int gh,
+                                                        int gw, int C, int act, int BR) {
+  constexpr int VN = Vec16<T>::N;           // elements per 16-byte chunk
+  constexpr int TPT = CONV_GROUP / VN;      // threads (chunks) per token
+  constexpr int NL = 256 / TPT;             // tokens per pass
+  extern __shared__ __align__(16) uint8_t cdyn[];
+  float* wt = reinterpret_cast<float*>(cdyn);  // [9][CONV_GROUP]
+  uint8_t* bufs = cdyn + 9 * CONV_GROUP * sizeof(float);
+  const size_t bb = conv_band_bytes(BR, gw, (int)sizeof(T));
+  const int g0 = blockIdx.x * CONV_GROUP;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < 9 * CONV_GROUP; i += 256) {
+    const int k = i / CONV_GROUP, c = i % CONV_GROUP;
+    wt[k * CONV_GROUP + c] = (g0 + c < C) ? taps[(g0 + c) * 9 + k] : 0.f;
+  }
+  const int chunk = tid % TPT, tl = tid / TPT;
+  const int c0 = g0 + chunk * VN;
+  const int ntok = gh * gw, nbands = (gh + BR - 1) / BR;
+  __syncthreads();
+  float wr[9][VN];  // this thread's taps, kept in registers for all its outputs
+#pragma unroll
+  for (int k = 0; k < 9; ++k)
+#pragma unroll
+    for (int i = 0; i < VN; ++i) wr[k][i] = wt[k * CONV_GROUP + chunk * VN + i];
+  const int rowchunks = gw * TPT;
+  for (int n = blockIdx.y; n < N; n += gridDim.y) {
+    const int64_t frame0 = (int64_t)n * ntok;
+    auto issue = [&](int bi, uint8_t* buf) {
+      const int y0 = bi * BR - 1;
+      for (int idx = tid; idx < (BR + 2) * rowchunks; idx += 256) {
+        const int r = idx / rowchunks, rem = idx % rowchunks, x = rem / TPT, k = rem % TPT;
+        const int yy = y0 + r, ch = g0 + k * VN;
+        const bool in = yy >= 0 && yy < gh && ch < C;
+        const T* src = in ? V + (frame0 + (int64_t)yy * gw + x) * ldv + ch : V;
+        cp_async16_cg(buf + (size_t)idx * 16, src, in ? 16u : 0u);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    __syncthreads();  // taps written; the previous frame's buffers are no longer read
+    issue(0, bufs);
+    for (int bi = 0; bi < nbands; ++bi) {
+      uint8_t* cur = bufs + (bi & 1) * bb;
+      if (bi + 1 < nbands) {
+        issue(bi + 1, bufs + ((bi + 1) & 1) * bb);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      }
+      __syncthreads();
+      const int y0 = bi * BR, rows = min(BR, gh - y0);
+      if (c0 < C) {
+        for (int p = tl; p < rows * gw; p += NL) {
+          const int ry = p / gw, x = p % gw;  // output row y0 + ry; its input rows are ry .. ry + 2 in the band
+          float acc[VN];
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+#pragma unroll
+          for (int dy = 0; dy < 3; ++dy) {
+#pragma unroll
+            for (int dx = -1; dx <= 1; ++dx) {
+              const int xx = x + dx;
+              if (xx < 0 || xx >= gw) continue;
+              float v[VN];
+              load16(reinterpret_cast<const T*>(cur + ((size_t)((ry + dy) * gw + xx) * TPT + chunk) * 16), v);
+#pragma unroll
+              for (int i = 0; i < VN; ++i) acc[i] = fmaf(wr[dy * 3 + dx + 1][i], v[i], acc[i]);
+            }
+          }
+          if (act == 1) {
+#pragma unroll
+            for (int i = 0; i < VN; ++i) acc[i] = acc[i] / (1.0f + expf(-acc[i]));
+          }
+          store16(out + (frame0 + (int64_t)(y0 + ry) * gw + x) * ldo + c0, acc);
+        }
+      }
+      __syncthreads();  // `cur` may be refilled by the prefetch of band bi + 2
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Low-precision copies of the fp32 fast weights, laid out for the tensor-core kernels:
 //   Wsh (bf16, apply) and Wsh16 (fp16, gradient) rows [0, Hm): W1 [H][m][d];

@@ -300,6 +300,53 @@ int launch_rownorm_any(const void* X, int64_t ld, int64_t rows, const ttt_dims& 
   return launch_rownorm<float>((float*)X, ld, rows, d, r_out, 0, s);
 }
 
+// ShortConv2D launch: the banded shared-memory kernel with the largest band
+// that keeps two CTAs per SM (or one, for very wide frames); the direct kernel
+// for frames too wide for one band of three rows.
+int launch_conv_any(const void* V, int64_t ldv, void* Vout, int64_t ldo, const float* taps, int64_t N, int gh, int gw,
+                    int C, int act, ttt_dtype dt, cudaStream_t s) {
+  if (N == 0) return TTT_OK;
+  const int esz = dt == TTT_BF16 ? 2 : 4;
+  const size_t row = (size_t)gw * CONV_GROUP * esz, fixed = 9 * CONV_GROUP * sizeof(float);
+  int BR = 0;
+  for (size_t budget : {(size_t)110 * 1024, (size_t)220 * 1024}) {
+    const int64_t br = (int64_t)((budget - fixed) / (2 * row)) - 2;
+    if (br >= 1) {
+      BR = (int)std::min<int64_t>(br, gh);
+      break;
+    }
+  }
+  const dim3 grid((C + CONV_GROUP - 1) / CONV_GROUP, (unsigned)std::min<int64_t>(N, 65535));
+  ProfScope ps(TTT_PROF_CONV, s);
+  if (BR >= 1) {
+    const size_t smem = conv_band_smem(BR, gw, esz);
+    if (dt == TTT_BF16) {
+      TTT_CHECK(cudaFuncSetAttribute(k_shortconv_band<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem));
+      k_shortconv_band<__nv_bfloat16><<<grid, 256, smem, s>>>((const __nv_bfloat16*)V, ldv, (__nv_bfloat16*)Vout, ldo,
+                                                              taps, (int)N, gh, gw, C, act, BR);
+    } else {
+      TTT_CHECK(cudaFuncSetAttribute(k_shortconv_band<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      k_shortconv_band<float><<<grid, 256, smem, s>>>((const float*)V, ldv, (float*)Vout, ldo, taps, (int)N, gh, gw, C,
+                                                      act, BR);
+    }
+  } else {
+    const int vn = dt == TTT_BF16 ? 8 : 4;
+    const int gv = CONV_GROUP / vn;
+    const dim3 block(gv, 256 / gv);
+    const dim3 grid2((unsigned)N, (C + CONV_GROUP - 1) / CONV_GROUP);
+    if (N > 2147483647) return TTT_ERR_UNSUPPORTED;
+    if (dt == TTT_BF16)
+      k_shortconv<__nv_bfloat16><<<grid2, block, 0, s>>>((const __nv_bfloat16*)V, ldv, (__nv_bfloat16*)Vout, ldo, taps,
+                                                         (int)N, gh, gw, C, act);
+    else
+      k_shortconv<float><<<grid2, block, 0, s>>>((const float*)V, ldv, (float*)Vout, ldo, taps, (int)N, gh, gw, C,
+                                                 act);
+  }
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
 int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStream_t s) {
   const int64_t n = (int64_t)d.heads * d.m * d.d;
   ProfScope ps(TTT_PROF_SHADOW, s);
@@ -592,19 +639,7 @@ HostLayout host_layout(const ttt_dims& d, int64_t T, ttt_dtype dt, bool conv) {
 
 int launch_conv(const void* V, void* Vout, const float* taps, int64_t frames, int gh, int gw, int C, ttt_dtype dt,
                 cudaStream_t s) {
-  if (frames == 0) return TTT_OK;
-  const int vn = dt == TTT_BF16 ? 8 : 4;
-  const int gv = CONV_GROUP / vn;
-  const dim3 block(gv, 256 / gv);
-  const dim3 grid((unsigned)frames, (C + CONV_GROUP - 1) / CONV_GROUP);
-  ProfScope ps(TTT_PROF_CONV, s);
-  if (dt == TTT_BF16)
-    k_shortconv<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)V, C, (__nv_bfloat16*)Vout, C, taps,
-                                                      (int)frames, gh, gw, C, 0);
-  else
-    k_shortconv<float><<<grid, block, 0, s>>>((const float*)V, C, (float*)Vout, C, taps, (int)frames, gh, gw, C, 0);
-  TTT_LAUNCHED();
-  return TTT_OK;
+  return launch_conv_any(V, C, Vout, C, taps, frames, gh, gw, C, 0, dt, s);
 }
 
 }  // namespace
@@ -652,19 +687,7 @@ int ttt_shortconv2d(const void* V, int64_t ld_v, void* Vout, int64_t ld_out, con
   if (!V || !Vout || !taps || V == Vout) return TTT_ERR_INVALID;
   if (!aligned16(V) || !aligned16(Vout) || (ld_v * (int64_t)esize(dtype)) % 16 || (ld_out * (int64_t)esize(dtype)) % 16)
     return TTT_ERR_ALIGN;
-  cudaStream_t s = (cudaStream_t)stream;
-  const int vn = dtype == TTT_BF16 ? 8 : 4;
-  const int gv = CONV_GROUP / vn;
-  const dim3 block(gv, 256 / gv);
-  const dim3 grid(N, (C + CONV_GROUP - 1) / CONV_GROUP);
-  ProfScope ps(TTT_PROF_CONV, s);
-  if (dtype == TTT_BF16)
-    k_shortconv<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)V, ld_v, (__nv_bfloat16*)Vout, ld_out, taps,
-                                                      N, h, w, C, act);
-  else
-    k_shortconv<float><<<grid, block, 0, s>>>((const float*)V, ld_v, (float*)Vout, ld_out, taps, N, h, w, C, act);
-  TTT_LAUNCHED();
-  return TTT_OK;
+  return launch_conv_any(V, ld_v, Vout, ld_out, taps, N, h, w, C, act, dtype, (cudaStream_t)stream);
 }
 
 int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, ttt_dims dims,
