@@ -201,7 +201,7 @@ __device__ __forceinline__ void store16_h(__half* p, const float (&v)[8]) {
   *reinterpret_cast<uint4*>(p) = x;
 }
 
-__global__ void __launch_bounds__(256, 2) k_prep_kv(const __nv_bfloat16* __restrict__ K, int64_t ldk,
+__global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restrict__ K, int64_t ldk,
                                                     const __nv_bfloat16* __restrict__ V, int64_t ldv,
                                                     __half* __restrict__ Kh, __half* __restrict__ Vh, int64_t rows,
                                                     int H, int d, int l2norm) {
@@ -215,15 +215,16 @@ __global__ void __launch_bounds__(256, 2) k_prep_kv(const __nv_bfloat16* __restr
     const __nv_bfloat16* krow = K + t * ldk;
     const __nv_bfloat16* vrow = V + t * ldv;
     if (nvt <= 32 * RN_MAX_VEC) {
-      float x[RN_MAX_VEC][VN], y[RN_MAX_VEC][VN];
+      // the row stays packed (bf16) in registers: small footprint, many tokens in flight per SM
+      uint4 xk[RN_MAX_VEC], xv[RN_MAX_VEC];
       int hv[RN_MAX_VEC];
 #pragma unroll
       for (int k = 0; k < RN_MAX_VEC; ++k) {
         const int v = lane + 32 * k;
         hv[k] = v < nvt ? v * VN / d : -1;
         if (hv[k] >= 0) {
-          load16(krow + v * VN, x[k]);
-          load16(vrow + v * VN, y[k]);
+          xk[k] = __ldg(reinterpret_cast<const uint4*>(krow + v * VN));
+          xv[k] = __ldg(reinterpret_cast<const uint4*>(vrow + v * VN));
         }
       }
       float inv[RN_MAX_VEC];
@@ -235,8 +236,12 @@ __global__ void __launch_bounds__(256, 2) k_prep_kv(const __nv_bfloat16* __restr
         for (int k = 0; k < RN_MAX_VEC; ++k) {
           ss[k] = 0.f;
           if (hv[k] >= 0) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&xk[k]);
 #pragma unroll
-            for (int i = 0; i < VN; ++i) ss[k] = fmaf(x[k][i], x[k][i], ss[k]);
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(h2[i]);
+              ss[k] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss[k]));
+            }
           }
         }
         for (int h = 0; h < H; ++h) {
@@ -253,10 +258,19 @@ __global__ void __launch_bounds__(256, 2) k_prep_kv(const __nv_bfloat16* __restr
 #pragma unroll
       for (int k = 0; k < RN_MAX_VEC; ++k)
         if (hv[k] >= 0) {
+          const __nv_bfloat162* hk = reinterpret_cast<const __nv_bfloat162*>(&xk[k]);
+          const __nv_bfloat162* hvv = reinterpret_cast<const __nv_bfloat162*>(&xv[k]);
+          uint4 ok, ov;
+          uint32_t* pk = reinterpret_cast<uint32_t*>(&ok);
+          uint32_t* pv = reinterpret_cast<uint32_t*>(&ov);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) x[k][i] *= inv[k];
-          store16_h(Kh + t * HD + (lane + 32 * k) * VN, x[k]);
-          store16_h(Vh + t * HD + (lane + 32 * k) * VN, y[k]);
+          for (int i = 0; i < 4; ++i) {
+            const float2 fk = __bfloat1622float2(hk[i]), fv = __bfloat1622float2(hvv[i]);
+            pk[i] = pack_f16x2(fk.x * inv[k], fk.y * inv[k]);
+            pv[i] = pack_f16x2(fv.x, fv.y);
+          }
+          *reinterpret_cast<uint4*>(Kh + t * HD + (lane + 32 * k) * VN) = ok;
+          *reinterpret_cast<uint4*>(Vh + t * HD + (lane + 32 * k) * VN) = ov;
         }
     } else {
       for (int h = 0; h < H; ++h) {

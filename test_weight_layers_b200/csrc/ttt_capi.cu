@@ -359,7 +359,7 @@ int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStre
 int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, int64_t T, const ttt_dims& d, int l2norm,
                    const Ws& w, cudaStream_t s) {
   if (T == 0) return TTT_OK;
-  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 8));
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 16));
   ProfScope ps(TTT_PROF_NORM, s);
   k_prep_kv<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, w.kh16, w.vh16, T,
                                    d.heads, d.d, l2norm);
