@@ -571,187 +571,156 @@ __device__ __forceinline__ float sum_parts(const float* parts) {
   return s;
 }
 
-__global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, const float* __restrict__ parts, int H,
-                          int d, int m, float eps) {
-  const int b = blockIdx.y;
+// X_b = orient(G_b) / (||G_b||_F + eps) in the wide orientation (r x c) and its
+// transpose XT_b (c x r), both written coalesced through a 32x32 shared tile.
+// grid (ceil(C/32), ceil(R/32), 3H) over G_b's own shape (R, C); block (32, 8).
+__global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, float* __restrict__ XT,
+                          const float* __restrict__ parts, int H, int d, int m, float eps) {
+  __shared__ float tile[32][33];
+  const int b = blockIdx.z;
   int R, C;
   mat_shape(b, H, d, m, R, C);
   const bool tall = R > C;
   const int64_t n = (int64_t)m * d;
   const float sc = 1.0f / (sqrtf(sum_parts(parts + b * NORM_PARTS)) + eps);
   const float* g = G + (int64_t)b * n;
-  float* x = X + (int64_t)b * n;
-  const int c = tall ? R : C;  // columns of X
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    // i indexes X (r, c) row-major
-    const int64_t xi = i / c, xj = i % c;
-    x[i] = (tall ? g[xj * C + xi] : g[i]) * sc;
-  }
-}
-
-// Delta in W's orientation: D_b = X_b for wide matrices, X_b^T for tall ones (32x32 smem tiles).
-// grid (ceil(C/32), ceil(R/32), 3H) over W's shape (R, C); block (32, 8).
-__global__ void k_ns_finish(const float* __restrict__ X, float* __restrict__ D, int H, int d, int m) {
-  __shared__ float tile[32][33];
-  const int b = blockIdx.z;
-  int R, C;
-  mat_shape(b, H, d, m, R, C);
-  const int64_t n = (int64_t)m * d;
-  const float* x = X + (int64_t)b * n;
-  float* o = D + (int64_t)b * n;
+  // the copy with G's layout: X (wide) or XT (tall); the transposed copy: the other
+  float* same = (tall ? XT : X) + (int64_t)b * n;
+  float* trans = (tall ? X : XT) + (int64_t)b * n;
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   if (r0 >= R || c0 >= C) return;
-  if (R <= C) {
-    for (int yy = threadIdx.y; yy < 32; yy += 8) {
-      const int r = r0 + yy, c = c0 + threadIdx.x;
-      if (r < R && c < C) o[(int64_t)r * C + c] = x[(int64_t)r * C + c];
-    }
-    return;
-  }
-  // tall: X is (C, R); D[r][c] = X[c][r]
   for (int yy = threadIdx.y; yy < 32; yy += 8) {
-    const int xc = c0 + yy, xr = r0 + threadIdx.x;  // X row xc, column xr
-    tile[yy][threadIdx.x] = (xc < C && xr < R) ? x[(int64_t)xc * R + xr] : 0.f;
+    const int r = r0 + yy, c = c0 + threadIdx.x;
+    float v = 0.f;
+    if (r < R && c < C) {
+      v = g[(int64_t)r * C + c] * sc;
+      same[(int64_t)r * C + c] = v;
+    }
+    tile[yy][threadIdx.x] = v;
   }
   __syncthreads();
   for (int yy = threadIdx.y; yy < 32; yy += 8) {
-    const int r = r0 + yy, c = c0 + threadIdx.x;
-    if (r < R && c < C) o[(int64_t)r * C + c] = tile[threadIdx.x][yy];
+    const int c = c0 + yy, r = r0 + threadIdx.x;  // trans is (C x R)
+    if (c < C && r < R) trans[(int64_t)c * R + r] = tile[threadIdx.x][yy];
   }
 }
 
 // ---- fp32 64x64 tile products of the Newton-Schulz iteration (CUDA cores)
+//
+// Every product is C = A B with both operands available as rows k: A^T rows
+// (A^T [K][M]; for the Gram, X^T; for A A and B X, the symmetric left factor
+// itself) and B rows ([K][N]).  A tile stages both [K][64] slabs (K <= NSC_KMAX
+// at a time) in shared memory with 16-byte asynchronous copies, all in flight
+// together, then each k step reads one float4 of A and one of B: 3 shared-memory
+// wavefronts per warp per 16 FMAs, so the FMAs, not shared memory, set the pace.
 
-constexpr int NSC_KMAX = 192;            // K extent staged in shared memory at once
-constexpr int NSC_SA = NSC_KMAX + 4;     // row stride of the staged A tile (floats)
-
-// dynamic shared memory: A tile [64][NSC_SA] then the B tile, [NSC_KMAX][64] or
-// (B = X^T) [64][NSC_SA]
-constexpr int NSC_B_FLOATS = 64 * NSC_SA > NSC_KMAX * 64 ? 64 * NSC_SA : NSC_KMAX * 64;
-constexpr int NSC_DYN_BYTES = (64 * NSC_SA + NSC_B_FLOATS) * 4;
+constexpr int NSC_KMAX = 192;  // K extent staged in shared memory at once
+// dynamic shared memory: A^T slab [NSC_KMAX][64] then B slab [NSC_KMAX][64]
+constexpr int NSC_DYN_BYTES = 2 * NSC_KMAX * 64 * 4;
 
 // 16-byte asynchronous global -> shared copy; src_bytes = 0 fills zeros
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+
+// rows k0 .. k0 + K - 1, columns c0 .. c0 + 63 of the row-major src (ld floats;
+// columns >= Cv read as 0) into dst[k][64]
+__device__ __forceinline__ void nsc_stage(const float* __restrict__ src, int ld, int c0, int Cv, int k0, int K,
+                                          float* dst) {
+  for (int idx = threadIdx.x; idx < K * 16; idx += 256) {
+    const int k = idx >> 4, q = idx & 15;
+    const bool in = c0 + 4 * q < Cv;
+    cp_async16(dst + k * 64 + 4 * q, src + (int64_t)(k0 + k) * ld + (in ? c0 + 4 * q : 0), in ? 16u : 0u);
+  }
 }
 
-// Tile column of acc[.][j] for thread column tx (see nsc_tile).
-__device__ __forceinline__ int nsc_col(int tx, int j, bool bt) { return bt ? tx + 16 * j : 4 * tx + j; }
-
-// acc += A(m0 + i, k0 + k) B(k0 + k, n0 + j) over k < K (K <= NSC_KMAX, K % 4 == 0)
-// for the 64x64 tile; thread (ty, tx) = (tid / 16, tid % 16) owns rows 4 ty ..
-// 4 ty + 3 and columns nsc_col(tx, 0..3, BT).  Both operands are staged whole in
-// shared memory by 16-byte asynchronous copies all in flight together (one L2
-// round trip per tile), then the FMAs run from shared memory.  A: rows of the
-// row-major matrix a (lda), rows >= Mv read as 0.  B (BT = false): rows k of
-// the row-major matrix bsrc (ldb), columns >= Nv read as 0; BT = true:
-// B(k, j) = bsrc[(n0 + j) ldb + k0 + k] (B = X^T), staged as rows j.
-// Leading dimensions and k0 are multiples of 4 floats.
-template <bool BT>
-__device__ __forceinline__ void nsc_tile(const float* __restrict__ a, int lda, int m0, int Mv,
-                                         const float* __restrict__ bsrc, int ldb, int n0, int Nv, int k0, int K,
+// acc += sum over k < K of A(m0 + i, k0 + k) B(k0 + k, n0 + j) for the 64x64 tile, with
+// at = A^T rows (lda; rows of length >= Mv) and b = B rows (ldb; length >= Nv).
+// Thread (ty, tx) = (tid / 16, tid % 16) owns rows 4 ty .. 4 ty + 3 and columns
+// 4 tx .. 4 tx + 3.  K <= NSC_KMAX; leading dimensions and column offsets are
+// multiples of 4 floats.
+__device__ __forceinline__ void nsc_tile(const float* __restrict__ at, int lda, int m0, int Mv,
+                                         const float* __restrict__ b, int ldb, int n0, int Nv, int k0, int K,
                                          float (&acc)[4][4], float* smA, float* smB) {
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int kq = K / 4;
   __syncthreads();  // the previous tile's reads of smA / smB are done
-  for (int idx = tid; idx < 64 * kq; idx += 256) {
-    const int row = idx / kq, q = idx % kq;
-    const bool in = m0 + row < Mv;
-    cp_async16(smA + row * NSC_SA + 4 * q, a + (int64_t)(in ? m0 + row : 0) * lda + k0 + 4 * q, in ? 16u : 0u);
-  }
-  if (!BT) {
-    for (int idx = tid; idx < K * 16; idx += 256) {
-      const int k = idx >> 4, q = idx & 15;
-      const bool in = n0 + 4 * q < Nv;
-      cp_async16(smB + k * 64 + 4 * q, bsrc + (int64_t)(k0 + k) * ldb + (in ? n0 + 4 * q : 0), in ? 16u : 0u);
-    }
-  } else {
-    // B^T: rows n0 + j of bsrc, stored like A ([64][NSC_SA])
-    for (int idx = tid; idx < 64 * kq; idx += 256) {
-      const int row = idx / kq, q = idx % kq;
-      const bool in = n0 + row < Nv;
-      cp_async16(smB + row * NSC_SA + 4 * q, bsrc + (int64_t)(in ? n0 + row : 0) * ldb + k0 + 4 * q, in ? 16u : 0u);
-    }
-  }
-  cp_async_wait_all();
+  nsc_stage(at, lda, m0, Mv, k0, K, smA);
+  nsc_stage(b, ldb, n0, Nv, k0, K, smB);
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  const float* ar = smA + (ty * 4) * NSC_SA;
-  if (!BT) {
 #pragma unroll 8
-    for (int k = 0; k < K; ++k) {
-      const float a4[4] = {ar[k], ar[NSC_SA + k], ar[2 * NSC_SA + k], ar[3 * NSC_SA + k]};
-      const float4 bv = *reinterpret_cast<const float4*>(smB + k * 64 + tx * 4);
-      const float b4[4] = {bv.x, bv.y, bv.z, bv.w};
+  for (int k = 0; k < K; ++k) {
+    const float4 av = *reinterpret_cast<const float4*>(smA + k * 64 + ty * 4);
+    const float4 bv = *reinterpret_cast<const float4*>(smB + k * 64 + tx * 4);
+    const float a4[4] = {av.x, av.y, av.z, av.w};
+    const float b4[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
-    }
-  } else {
-    // columns tx, tx + 16, tx + 32, tx + 48 (conflict-free reads of the row-stored B^T)
-    const float* br = smB + tx * NSC_SA;
-#pragma unroll 8
-    for (int k = 0; k < K; ++k) {
-      const float a4[4] = {ar[k], ar[NSC_SA + k], ar[2 * NSC_SA + k], ar[3 * NSC_SA + k]};
-      const float b4[4] = {br[k], br[16 * NSC_SA + k], br[32 * NSC_SA + k], br[48 * NSC_SA + k]};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
-    }
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
   }
 }
 
-// Batched C = alpha * A * B + beta * Cin, fp32, one 64x64 output tile per CTA
-// (256 threads), K staged in shared memory in pieces of NSC_KMAX.  A [M][K]
-// (lda), B [K][N] (ldb); leading dimensions and K are multiples of 4.
-// Dynamic shared memory: NSC_DYN_BYTES.
-__global__ void __launch_bounds__(256) k_gemm_f32(int M, int N, int K, const float* __restrict__ A, int lda,
-                                                  int64_t sA, const float* __restrict__ B, int ldb, int64_t sB,
-                                                  float* __restrict__ C, int ldc, int64_t sC,
+// Batched C = alpha S B + beta Cin with S symmetric (M x M, so the rows of S
+// serve as rows of S^T), B [M][N] (ldb), one 64x64 output tile per CTA.  With
+// CT != null the tile is also written transposed to CT [N][M] (through shared
+// memory, so both stores are coalesced).  Dynamic shared memory: NSC_DYN_BYTES.
+__global__ void __launch_bounds__(256) k_gemm_sym(int M, int N, const float* __restrict__ S, int64_t sS,
+                                                  const float* __restrict__ B, int ldb, int64_t sB,
+                                                  float* __restrict__ C, int ldc, int64_t sC, float* __restrict__ CT,
                                                   const float* __restrict__ Cin, float alpha, float beta) {
   extern __shared__ __align__(16) float gemm_dyn[];
   float* smA = gemm_dyn;
-  float* smB = gemm_dyn + 64 * NSC_SA;
+  float* smB = gemm_dyn + NSC_KMAX * 64;
   const int b = blockIdx.z;
-  A += b * sA;
+  S += b * sS;
   B += b * sB;
   C += b * sC;
+  if (CT) CT += b * sC;
   if (Cin) Cin += b * sC;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float acc[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += NSC_KMAX)
-    nsc_tile<false>(A, lda, m0, M, B, ldb, n0, N, k0, min(NSC_KMAX, K - k0), acc, smA, smB);
+  for (int k0 = 0; k0 < M; k0 += NSC_KMAX)
+    nsc_tile(S, M, m0, M, B, ldb, n0, N, k0, min(NSC_KMAX, M - k0), acc, smA, smB);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int gm = m0 + ty * 4 + i, gn = n0 + nsc_col(tx, j, false);
-      if (gm < M && gn < N) {
-        float v = alpha * acc[i][j];
-        if (Cin) v = fmaf(beta, Cin[(int64_t)gm * ldc + gn], v);
-        C[(int64_t)gm * ldc + gn] = v;
-      }
+      const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
+      float v = alpha * acc[i][j];
+      if (Cin && gm < M && gn < N) v = fmaf(beta, Cin[(int64_t)gm * ldc + gn], v);
+      acc[i][j] = v;
+      if (gm < M && gn < N) C[(int64_t)gm * ldc + gn] = v;
     }
+  if (CT) {
+    float* tt = smA;  // [64][65]; the staging slabs are no longer read
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tt[(tx * 4 + j) * 65 + ty * 4 + i] = acc[i][j];
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * 64; e += 256) {
+      const int nn = e >> 6, mm = e & 63;  // CT row n0 + nn, column m0 + mm
+      if (n0 + nn < N && m0 + mm < M) CT[(int64_t)(n0 + nn) * M + m0 + mm] = tt[nn * 65 + mm];
+    }
+  }
 }
 
-// Gram matrices A_b = X_b X_b^T for the Newton-Schulz batch: upper-triangular
+// Gram matrices A_b = X_b X_b^T from X^T (c x r, row-major): upper-triangular
 // 64x64 tiles only (A is symmetric), split-K over NS_GRAM_SPLIT slices of the
 // long dimension for parallelism.  grid (tiles, NS_GRAM_SPLIT, batch); partial
 // P[s][b][i][j] for the tile's (i, j); k_gram_reduce sums the slices in fixed
 // order and mirrors the lower triangle.  Dynamic shared memory: NSC_DYN_BYTES.
 constexpr int NS_GRAM_SPLIT = 4;
 
-__global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float* __restrict__ X, int64_t sX,
+__global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float* __restrict__ XT, int64_t sX,
                                                       float* __restrict__ P) {
   extern __shared__ __align__(16) float gram_dyn[];
   float* smA = gram_dyn;
-  float* smB = gram_dyn + 64 * NSC_SA;
+  float* smB = gram_dyn + NSC_KMAX * 64;
   const int rt = (r + 63) / 64;
   // tile index -> (ti <= tj) in row-major upper-triangular order
   int t = blockIdx.x, ti = 0;
@@ -760,18 +729,18 @@ __global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float*
   const int s = blockIdx.y, b = blockIdx.z;
   const int kper = ((c + NS_GRAM_SPLIT - 1) / NS_GRAM_SPLIT + 15) / 16 * 16;
   const int k_begin = s * kper, k_end = min(c, k_begin + kper);
-  const float* x = X + (int64_t)b * sX;
+  const float* xt = XT + (int64_t)b * sX;
   const int m0 = ti * 64, n0 = tj * 64;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float acc[4][4] = {};
   for (int k0 = k_begin; k0 < k_end; k0 += NSC_KMAX)
-    nsc_tile<true>(x, c, m0, r, x, c, n0, r, k0, min(NSC_KMAX, k_end - k0), acc, smA, smB);
+    nsc_tile(xt, r, m0, r, xt, r, n0, r, k0, min(NSC_KMAX, k_end - k0), acc, smA, smB);
   float* out = P + ((int64_t)s * gridDim.z + b) * (int64_t)r * r;
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int gm = m0 + ty * 4 + i, gn = n0 + nsc_col(tx, j, true);
+      const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
       if (gm < r && gn < r) out[(int64_t)gm * r + gn] = acc[i][j];
     }
 }
@@ -792,21 +761,29 @@ __global__ void k_gram_reduce(int r, int nb, const float* __restrict__ P, float*
 
 // ---------------------------------------------------------------------------
 // Muon weight step (ZipMap key design 3): W <- ||W|| (W - lr D) / ||W - lr D||,
-// D in W's orientation (k_ns_finish), or G itself when Newton-Schulz is off.
+// Delta in W's orientation: X_b (r x c) for a wide W_b, XT_b for a tall one
+// (Dw = X, Dt = XT), or G itself when Newton-Schulz is off (Dw = Dt = G).
 
 __device__ __forceinline__ float* mat_ptr(float* W1, float* W3, float* W2, int b, int H, int64_t n) {
   return b < H ? W1 + (int64_t)b * n : (b < 2 * H ? W3 + (int64_t)(b - H) * n : W2 + (int64_t)(b - 2 * H) * n);
 }
 
 // partials out[(b * NORM_PARTS + p) * 2 + {0,1}] of ||W_b||^2 and ||W_b - lr D_b||^2
-__global__ void __launch_bounds__(256) k_step_partials(float* W1, float* W3, float* W2, const float* __restrict__ D,
-                                                       int H, int d, int m, float lr, float* __restrict__ out) {
+__device__ __forceinline__ const float* delta_of(const float* Dw, const float* Dt, int b, int H, int d, int m) {
+  int R, C;
+  mat_shape(b, H, d, m, R, C);
+  return (R > C ? Dt : Dw) + (int64_t)b * m * d;
+}
+
+__global__ void __launch_bounds__(256) k_step_partials(float* W1, float* W3, float* W2, const float* __restrict__ Dw,
+                                                       const float* __restrict__ Dt, int H, int d, int m, float lr,
+                                                       float* __restrict__ out) {
   __shared__ float red[9];
   const int b = blockIdx.x, p = blockIdx.y;
   const int64_t n = (int64_t)m * d, n4 = n / 4, per = (n4 + NORM_PARTS - 1) / NORM_PARTS;
   const int64_t i0 = p * per, i1 = min(n4, i0 + per);
   const float4* w = reinterpret_cast<const float4*>(mat_ptr(W1, W3, W2, b, H, n));
-  const float4* dl = reinterpret_cast<const float4*>(D + (int64_t)b * n);
+  const float4* dl = reinterpret_cast<const float4*>(delta_of(Dw, Dt, b, H, d, m));
   float s0 = 0.f, s1 = 0.f;
   for (int64_t i = i0 + threadIdx.x; i < i1; i += 256) {
     const float4 a = w[i], q = dl[i];
@@ -822,12 +799,12 @@ __global__ void __launch_bounds__(256) k_step_partials(float* W1, float* W3, flo
   }
 }
 
-__global__ void k_step_apply(float* W1, float* W3, float* W2, const float* __restrict__ D, int H, int d, int m, float lr,
-                             int renorm, const float* __restrict__ parts) {
+__global__ void k_step_apply(float* W1, float* W3, float* W2, const float* __restrict__ Dw, const float* __restrict__ Dt,
+                             int H, int d, int m, float lr, int renorm, const float* __restrict__ parts) {
   const int b = blockIdx.y;
   const int64_t n = (int64_t)m * d, n4 = n / 4;
   float4* w = reinterpret_cast<float4*>(mat_ptr(W1, W3, W2, b, H, n));
-  const float4* dl = reinterpret_cast<const float4*>(D + (int64_t)b * n);
+  const float4* dl = reinterpret_cast<const float4*>(delta_of(Dw, Dt, b, H, d, m));
   float sc = 1.f;
   if (renorm) {
     float s0 = 0.f, s1 = 0.f;

@@ -76,8 +76,10 @@ struct Ws {
   __nv_bfloat16* w2b;  // [H][d][m]
   float* G;            // [3][H*m*d]
   float* partial;      // [S_max][3][H*m*d]
-  float* X;            // [3H][m*d]
+  float* X;            // [3H][m*d] Newton-Schulz iterate, wide orientation (r x c)
   float* X2;           // [3H][m*d]
+  float* XT;           // [3H][m*d] its transpose (c x r)
+  float* XT2;          // [3H][m*d]
   float* A;            // [3H][r*r]
   float* B;            // [3H][r*r]
   float* gram;         // [NS_GRAM_SPLIT][3H][r*r] split-K partials of the Gram matrices
@@ -127,6 +129,8 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_p = take((size_t)w.s_max * 3 * n * 4);
   const size_t o_X = take(3 * n * 4);
   const size_t o_X2 = take(3 * n * 4);
+  const size_t o_XT = take(3 * n * 4);
+  const size_t o_XT2 = take(3 * n * 4);
   const size_t o_A = take(3 * H * r * r * 4);
   const size_t o_B = take(3 * H * r * r * 4);
   const size_t o_gram = take((size_t)NS_GRAM_SPLIT * 3 * H * r * r * 4);
@@ -148,6 +152,8 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
     w.partial = reinterpret_cast<float*>(b + o_p);
     w.X = reinterpret_cast<float*>(b + o_X);
     w.X2 = reinterpret_cast<float*>(b + o_X2);
+    w.XT = reinterpret_cast<float*>(b + o_XT);
+    w.XT2 = reinterpret_cast<float*>(b + o_XT2);
     w.A = reinterpret_cast<float*>(b + o_A);
     w.B = reinterpret_cast<float*>(b + o_B);
     w.gram = reinterpret_cast<float*>(b + o_gram);
@@ -457,40 +463,40 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
   const int64_t n = (int64_t)mm * dd;
   const int nb = 3 * H;
   const int r = std::min(mm, dd), c = std::max(mm, dd);
-  const float* D = G;
+  const float* Dw = G;
+  const float* Dt = G;
   ProfScope ps(TTT_PROF_NS, s);
   if (ns.iters > 0) {
     k_frob_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(G, n, w.norms);
     TTT_LAUNCHED();
-    k_ns_init<<<dim3(grid1d(n, 256) / nb + 1, nb), 256, 0, s>>>(G, w.X, w.norms, H, dd, mm, ns.eps);
+    k_ns_init<<<dim3((c + 31) / 32, (c + 31) / 32, nb), dim3(32, 8), 0, s>>>(G, w.X, w.XT, w.norms, H, dd, mm, ns.eps);
     TTT_LAUNCHED();
-    float* X = w.X;
-    float* X2 = w.X2;
+    float *X = w.X, *X2 = w.X2, *XT = w.XT, *XT2 = w.XT2;
     const int rt = (r + 63) / 64, ct = (c + 63) / 64;
     TTT_CHECK(cudaFuncSetAttribute(k_gram_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, NSC_DYN_BYTES));
-    TTT_CHECK(cudaFuncSetAttribute(k_gemm_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, NSC_DYN_BYTES));
+    TTT_CHECK(cudaFuncSetAttribute(k_gemm_sym, cudaFuncAttributeMaxDynamicSharedMemorySize, NSC_DYN_BYTES));
+    const int64_t rr = (int64_t)r * r;
     for (int it = 0; it < ns.iters; ++it) {
-      k_gram_partial<<<dim3(rt * (rt + 1) / 2, NS_GRAM_SPLIT, nb), 256, NSC_DYN_BYTES, s>>>(r, c, X, n, w.gram);
+      // A = X X^T (from X^T), B = b A + c A A, X' = a X + B X (and X'^T)
+      k_gram_partial<<<dim3(rt * (rt + 1) / 2, NS_GRAM_SPLIT, nb), 256, NSC_DYN_BYTES, s>>>(r, c, XT, n, w.gram);
       TTT_LAUNCHED();
-      k_gram_reduce<<<grid1d((int64_t)nb * r * r, 256), 256, 0, s>>>(r, nb, w.gram, w.A);
+      k_gram_reduce<<<grid1d((int64_t)nb * rr, 256), 256, 0, s>>>(r, nb, w.gram, w.A);
       TTT_LAUNCHED();
-      k_gemm_f32<<<dim3(rt, rt, nb), 256, NSC_DYN_BYTES, s>>>(r, r, r, w.A, r, (int64_t)r * r, w.A, r, (int64_t)r * r, w.B,
-                                                          r, (int64_t)r * r, w.A, ns.c, ns.b);
+      k_gemm_sym<<<dim3(rt, rt, nb), 256, NSC_DYN_BYTES, s>>>(r, r, w.A, rr, w.A, r, rr, w.B, r, rr, nullptr, w.A,
+                                                               ns.c, ns.b);
       TTT_LAUNCHED();
-      k_gemm_f32<<<dim3(ct, rt, nb), 256, NSC_DYN_BYTES, s>>>(r, c, r, w.B, r, (int64_t)r * r, X, c, n, X2, c, n, X, 1.f,
-                                                          ns.a);
+      k_gemm_sym<<<dim3(ct, rt, nb), 256, NSC_DYN_BYTES, s>>>(r, c, w.B, rr, X, c, n, X2, c, n, XT2, X, 1.f, ns.a);
       TTT_LAUNCHED();
       std::swap(X, X2);
+      std::swap(XT, XT2);
     }
-    // Delta back in W's orientation, into the buffer X does not occupy
-    k_ns_finish<<<dim3((c + 31) / 32, (c + 31) / 32, nb), dim3(32, 8), 0, s>>>(X, X2, H, dd, mm);
-    TTT_LAUNCHED();
-    D = X2;
+    Dw = X;
+    Dt = XT;
   }
-  k_step_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, w.stepn);
+  k_step_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(W.W1, W.W3, W.W2, Dw, Dt, H, dd, mm, ns.lr, w.stepn);
   TTT_LAUNCHED();
-  k_step_apply<<<dim3(grid1d(n / 4, 256) / nb + 1, nb), 256, 0, s>>>(W.W1, W.W3, W.W2, D, H, dd, mm, ns.lr, ns.renorm,
-                                                                    w.stepn);
+  k_step_apply<<<dim3(grid1d(n / 4, 256) / nb + 1, nb), 256, 0, s>>>(W.W1, W.W3, W.W2, Dw, Dt, H, dd, mm, ns.lr,
+                                                                    ns.renorm, w.stepn);
   TTT_LAUNCHED();
   return TTT_OK;
 }
