@@ -187,7 +187,10 @@ __global__ void __launch_bounds__(256, 4) k_rownorm(T* X, int64_t ld, int64_t ro
 // ---------------------------------------------------------------------------
 // Update-operand preparation: one pass over K and V that writes the fp16
 // operands of the tensor-core gradient kernel, K^ = k / max(||k||, 1e-12) per
-// head (or k itself) and V, densely [T][H*d].  bf16 -> fp16 is exact for values
+// head (or k itself) and V' = vscale * eta_(t,h) * v, densely [T][H*d].  The loss is
+// linear in v, so folding the per-token weight (and the gradient's fp16 scale)
+// into V is exact algebra: the forward then yields dL/du = -eta z directly and
+// the gradient of W2 needs no per-token scaling.  bf16 -> fp16 is exact for values
 // in fp16's normal range; fp16 carries three more significand bits than bf16,
 // which the chained Muon updates need.  One warp per token, the whole row loaded
 // before any reduction.
@@ -203,6 +206,7 @@ __device__ __forceinline__ void store16_h(__half* p, const float (&v)[8]) {
 
 __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restrict__ K, int64_t ldk,
                                                     const __nv_bfloat16* __restrict__ V, int64_t ldv,
+                                                    const float* __restrict__ eta, float vscale,
                                                     __half* __restrict__ Kh, __half* __restrict__ Vh, int64_t rows,
                                                     int H, int d, int l2norm) {
   constexpr int VN = 8;
@@ -218,6 +222,9 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
       // the row stays packed (bf16) in registers: small footprint, many tokens in flight per SM
       uint4 xk[RN_MAX_VEC], xv[RN_MAX_VEC];
       int hv[RN_MAX_VEC];
+      // eta of this token: lane h < H holds head h's weight (one load per token,
+      // issued with the row loads); the vectors fetch theirs by shuffle
+      const float eh = (lane < H) ? __ldg(eta + t * H + lane) : 0.f;
 #pragma unroll
       for (int k = 0; k < RN_MAX_VEC; ++k) {
         const int v = lane + 32 * k;
@@ -256,7 +263,8 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
         }
       }
 #pragma unroll
-      for (int k = 0; k < RN_MAX_VEC; ++k)
+      for (int k = 0; k < RN_MAX_VEC; ++k) {
+        const float vek = vscale * __shfl_sync(0xffffffffu, eh, hv[k] >= 0 ? hv[k] : 0);
         if (hv[k] >= 0) {
           const __nv_bfloat162* hk = reinterpret_cast<const __nv_bfloat162*>(&xk[k]);
           const __nv_bfloat162* hvv = reinterpret_cast<const __nv_bfloat162*>(&xv[k]);
@@ -267,11 +275,12 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
           for (int i = 0; i < 4; ++i) {
             const float2 fk = __bfloat1622float2(hk[i]), fv = __bfloat1622float2(hvv[i]);
             pk[i] = pack_f16x2(fk.x * inv[k], fk.y * inv[k]);
-            pv[i] = pack_f16x2(fv.x, fv.y);
+            pv[i] = pack_f16x2(fv.x * vek, fv.y * vek);
           }
           *reinterpret_cast<uint4*>(Kh + t * HD + (lane + 32 * k) * VN) = ok;
           *reinterpret_cast<uint4*>(Vh + t * HD + (lane + 32 * k) * VN) = ov;
         }
+      }
     } else {
       for (int h = 0; h < H; ++h) {
         float ss = 0.f;
@@ -283,12 +292,16 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
         }
         ss = warp_sum(ss);
         const float r = l2norm ? 1.0f / fmaxf(sqrtf(ss), 1e-12f) : 1.f;
+        const float ve = vscale * eta[t * H + h];
         for (int v = lane; v < d / VN; v += 32) {
           float x[VN], y[VN];
           load16(krow + h * d + v * VN, x);
           load16(vrow + h * d + v * VN, y);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) x[i] *= r;
+          for (int i = 0; i < VN; ++i) {
+            x[i] *= r;
+            y[i] *= ve;
+          }
           store16_h(Kh + t * HD + h * d + v * VN, x);
           store16_h(Vh + t * HD + h * d + v * VN, y);
         }

@@ -84,8 +84,8 @@ template <int D>
 __global__ void __launch_bounds__(UPD_THREADS, 1)
     k_update_grad_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
-                     const __grid_constant__ CUtensorMap tmW, const float* __restrict__ eta,
-                     float* __restrict__ partial, int64_t T, int H, int m,
+                     const __grid_constant__ CUtensorMap tmW, float* __restrict__ partial, int64_t T, int H,
+                     int m,
                      int tiles_total, int S, unsigned int* status, unsigned long long timeout_ns) {
   using L = UpdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -299,8 +299,6 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
-      const int64_t t = (int64_t)(t_begin + i) * TC_TILE + row;
-      const float e = (t < T) ? eta[t * H + h] : 0.f;
       if (!__all_sync(0xffffffffu, mbar_wait(fdone, i & 1, g))) { ok = false; break; }
       tc_fence_after();
       uint32_t a1[32], a3[32], az[32];
@@ -313,9 +311,10 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_n(ffree, 32);  // F may now be overwritten by the next tile's forward
-      // dH and U~ are stored as fp16 scaled by 2^8 (clear of fp16 subnormals); the
-      // gradient readout multiplies by 2^-8, which is exact
-      const float2 ne2 = make_float2(-e * GRAD_SCALE, -e * GRAD_SCALE);  // -eta (scaled)
+      // V arrives as -2^8 eta v (the preparation kernel folds the per-token
+      // weight into it), so Z = dL/du scaled by 2^8 (clear of fp16 subnormals) and
+      // dH is scaled the same way; U~ = u, and g2 = V'^T U~ carries the 2^8.  The
+      // gradient readout multiplies by 2^-8, which is exact.
       const float2 half2 = make_float2(0.5f, 0.5f);
       const float2 mhalf2 = make_float2(-0.5f, -0.5f);
       uint32_t p1[16], p3[16], pu[16];
@@ -330,11 +329,11 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
         const float2 oms = __ffma2_rn(th, mhalf2, half2);        // 1 - sigmoid(h1)
         const float2 a = __fmul2_rn(h1, s);                      // SiLU(h1)
         const float2 u = __fmul2_rn(a, h3);
-        const float2 dz = __fmul2_rn(ne2, z);                    // dL/du = -eta z
+        const float2 dz = z;                                     // dL/du = -eta z (scaled)
         const float2 qd = __ffma2_rn(a, oms, s);                 // SiLU'(h1) = s + a (1 - s)
         const float2 d1 = __fmul2_rn(__fmul2_rn(dz, h3), qd);    // dL/dh1
         const float2 d3 = __fmul2_rn(dz, a);                     // dL/dh3
-        const float2 ut = __fmul2_rn(ne2, u);                    // -eta u
+        const float2 ut = u;
         p1[j >> 1] = pack_f16x2(d1.x, d1.y);
         p3[j >> 1] = pack_f16x2(d3.x, d3.y);
         pu[j >> 1] = pack_f16x2(ut.x, ut.y);

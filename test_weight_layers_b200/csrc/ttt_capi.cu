@@ -361,14 +361,14 @@ int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStre
   return TTT_OK;
 }
 
-// fp16 gradient operands K^, V (dense [T][H*d]) from the caller's bf16 K, V
-int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, int64_t T, const ttt_dims& d, int l2norm,
-                   const Ws& w, cudaStream_t s) {
+// fp16 gradient operands K^ and V' = -2^8 eta v (dense [T][H*d]) from the caller's bf16 K, V
+int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta, int64_t T,
+                   const ttt_dims& d, int l2norm, const Ws& w, cudaStream_t s) {
   if (T == 0) return TTT_OK;
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 16));
   ProfScope ps(TTT_PROF_NORM, s);
-  k_prep_kv<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, w.kh16, w.vh16, T,
-                                   d.heads, d.d, l2norm);
+  k_prep_kv<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, -GRAD_SCALE,
+                                   w.kh16, w.vh16, T, d.heads, d.d, l2norm);
   TTT_LAUNCHED();
   return TTT_OK;
 }
@@ -381,12 +381,14 @@ struct UpdOperands {
   const float* rk;
 };
 
-// Operands of the gradient kernels for T tokens: fp16 K^/V copies in bf16 mode,
-// the caller's K/V plus per-token inverse norms in fp32 mode.
-int prepare_update_operands(const void* K, int64_t ldk, const void* V, int64_t ldv, int64_t T, const ttt_dims& d,
-                            ttt_dtype dt, int l2norm, const Ws& w, cudaStream_t s, UpdOperands* op) {
+// Operands of the gradient kernels for T tokens: fp16 K^/V' copies in bf16 mode
+// (V' carries the per-token weights eta), the caller's K/V plus per-token inverse
+// norms in fp32 mode.
+int prepare_update_operands(const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta, int64_t T,
+                            const ttt_dims& d, ttt_dtype dt, int l2norm, const Ws& w, cudaStream_t s,
+                            UpdOperands* op) {
   if (dt == TTT_BF16) {
-    TTT_TRY(launch_prep_kv(K, ldk, V, ldv, T, d, l2norm, w, s));
+    TTT_TRY(launch_prep_kv(K, ldk, V, ldv, eta, T, d, l2norm, w, s));
     const int64_t hd = (int64_t)d.heads * d.d;
     *op = {w.kh16, hd, w.vh16, hd, nullptr};
     return TTT_OK;
@@ -429,12 +431,12 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
     if (d.d == 192) {
       auto k = k_update_grad_tc<192>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<192>::ALLOC));
-      k<<<grid, UPD_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, w.partial, T, d.heads, d.m,
+      k<<<grid, UPD_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, w.partial, T, d.heads, d.m,
                                                           tiles, S, w.status, wait_timeout_ns());
     } else {
       auto k = k_update_grad_tc<128>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<128>::ALLOC));
-      k<<<grid, UPD_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, eta, w.partial, T, d.heads, d.m,
+      k<<<grid, UPD_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, w.partial, T, d.heads, d.m,
                                                           tiles, S, w.status, wait_timeout_ns());
     }
     TTT_LAUNCHED();
@@ -710,7 +712,7 @@ int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int6
   cudaStream_t s = (cudaStream_t)stream;
   Ws w = carve(ws, dims, T, dtype);
   UpdOperands op;
-  TTT_TRY(prepare_update_operands(K, ldk, V, ldv, T, dims, dtype, io->qk_l2norm, w, s, &op));
+  TTT_TRY(prepare_update_operands(K, ldk, V, ldv, eta, T, dims, dtype, io->qk_l2norm, w, s, &op));
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
   return run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, T, dims, dtype, w, G, s);
 }
@@ -741,7 +743,7 @@ int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, in
   cudaStream_t s = (cudaStream_t)stream;
   Ws w = carve(ws, dims, T, dtype);
   UpdOperands op;
-  TTT_TRY(prepare_update_operands(K, ldk, V, ldv, T, dims, dtype, io->qk_l2norm, w, s, &op));
+  TTT_TRY(prepare_update_operands(K, ldk, V, ldv, eta, T, dims, dtype, io->qk_l2norm, w, s, &op));
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
   for (int st = 0; st < steps; ++st) {
     TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, T, dims, dtype, w, w.G, s));
@@ -835,7 +837,7 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
     uint8_t* o = static_cast<uint8_t*>(O) + c0 * ldo * es;
     const float* e = eta + c0 * dims.heads;
     UpdOperands op;
-    TTT_TRY(prepare_update_operands(k, ldk, v, ldv, tc, dims, dtype, io->qk_l2norm, w, s, &op));
+    TTT_TRY(prepare_update_operands(k, ldk, v, ldv, e, tc, dims, dtype, io->qk_l2norm, w, s, &op));
     if (order == 0) TTT_TRY(run_apply(W, q, ldq, o, ldo, io->qk_l2norm, w.rq, tc, dims, dtype, w, s));
     for (int st = 0; st < steps; ++st) {
       TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, e, op.rk, tc, dims, dtype, w, w.G, s));
@@ -953,7 +955,8 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
         const uint8_t* v = vsrc(t0, tb);
         if (!v) return TTT_ERR_CUDA;
         UpdOperands op;
-        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, tb, dims, dtype, io->qk_l2norm, w, s, &op));
+        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, dEta + t0 * dims.heads, tb, dims, dtype,
+                                        io->qk_l2norm, w, s, &op));
         for (int st = 0; st < steps; ++st) {
           TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s));
           TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
@@ -976,7 +979,8 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
           wb.rk = w.rk + t0 * dims.heads;
         }
         UpdOperands op;
-        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, tb, dims, dtype, io->qk_l2norm, wb, s, &op));
+        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, dEta + t0 * dims.heads, tb, dims, dtype,
+                                        io->qk_l2norm, wb, s, &op));
         TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s,
                          b > 0));
       }
