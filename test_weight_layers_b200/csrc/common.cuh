@@ -35,6 +35,15 @@ __device__ __forceinline__ unsigned long long globaltimer() {
   return t;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start before the previous kernel on the stream has
+// finished; pdl_wait() blocks until that kernel has completed and its writes are
+// visible (it returns at once for a kernel launched normally).  pdl_trigger()
+// lets the next kernel start its own launch early, once every block of this one
+// has issued it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   uintptr_t a = reinterpret_cast<uintptr_t>(p);
   // shared-window addresses: align the shared offset, not the generic pointer

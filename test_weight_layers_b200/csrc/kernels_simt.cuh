@@ -494,6 +494,8 @@ __global__ void __launch_bounds__(256, 2) k_shortconv_band(const T* __restrict__
 __global__ void k_shadow(const float* __restrict__ W1, const float* __restrict__ W3, const float* __restrict__ W2,
                          __nv_bfloat16* __restrict__ Wsh, __nv_bfloat16* __restrict__ W2b, __half* __restrict__ Wsh16,
                          int H, int d, int m) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t n = (int64_t)H * m * d;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     Wsh[i] = __float2bfloat16_rn(W1[i]);
@@ -563,6 +565,8 @@ constexpr int NORM_PARTS = 16;  // slices per matrix for the norm reductions
 // partial sums of squares: out[b * NORM_PARTS + p] over slice p of matrix b (n_per % 4 == 0)
 __global__ void __launch_bounds__(256) k_frob_partials(const float* __restrict__ src, int64_t n_per,
                                                        float* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[9];
   const int b = blockIdx.x, p = blockIdx.y;
   const int64_t n4 = n_per / 4, per = (n4 + NORM_PARTS - 1) / NORM_PARTS;
@@ -589,6 +593,8 @@ __device__ __forceinline__ float sum_parts(const float* parts) {
 // grid (ceil(C/32), ceil(R/32), 3H) over G_b's own shape (R, C); block (32, 8).
 __global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, float* __restrict__ XT,
                           const float* __restrict__ parts, int H, int d, int m, float eps) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float tile[32][33];
   const int b = blockIdx.z;
   int R, C;
@@ -683,6 +689,8 @@ __global__ void __launch_bounds__(256) k_gemm_sym(int M, int N, const float* __r
                                                   const float* __restrict__ B, int ldb, int64_t sB,
                                                   float* __restrict__ C, int ldc, int64_t sC, float* __restrict__ CT,
                                                   const float* __restrict__ Cin, float alpha, float beta) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(16) float gemm_dyn[];
   float* smA = gemm_dyn;
   float* smB = gemm_dyn + NSC_KMAX * 64;
@@ -731,6 +739,8 @@ constexpr int NS_GRAM_SPLIT = 4;
 
 __global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float* __restrict__ XT, int64_t sX,
                                                       float* __restrict__ P) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(16) float gram_dyn[];
   float* smA = gram_dyn;
   float* smB = gram_dyn + NSC_KMAX * 64;
@@ -758,16 +768,17 @@ __global__ void __launch_bounds__(256) k_gram_partial(int r, int c, const float*
     }
 }
 
-// A[b][i][j] = sum_s P[s][b][min(i,j)][max(i,j)] (slices in fixed order)
-__global__ void k_gram_reduce(int r, int nb, const float* __restrict__ P, float* __restrict__ A) {
+// A[b][i][j] = sum_s P[s][b][min(i,j)][max(i,j)] over nsplit slices, in fixed order
+__global__ void k_gram_reduce(int r, int nb, int nsplit, const float* __restrict__ P, float* __restrict__ A) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t n = (int64_t)r * r;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * nb; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t b = e / n, ij = e % n;
     const int i = (int)(ij / r), j = (int)(ij % r);
     const int64_t src = b * n + (int64_t)min(i, j) * r + max(i, j);
     float acc = 0.f;
-#pragma unroll
-    for (int s = 0; s < NS_GRAM_SPLIT; ++s) acc += P[(int64_t)s * nb * n + src];
+    for (int s = 0; s < nsplit; ++s) acc += P[(int64_t)s * nb * n + src];
     A[e] = acc;
   }
 }
@@ -791,6 +802,8 @@ __device__ __forceinline__ const float* delta_of(const float* Dw, const float* D
 __global__ void __launch_bounds__(256) k_step_partials(float* W1, float* W3, float* W2, const float* __restrict__ Dw,
                                                        const float* __restrict__ Dt, int H, int d, int m, float lr,
                                                        float* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[9];
   const int b = blockIdx.x, p = blockIdx.y;
   const int64_t n = (int64_t)m * d, n4 = n / 4, per = (n4 + NORM_PARTS - 1) / NORM_PARTS;
@@ -814,6 +827,8 @@ __global__ void __launch_bounds__(256) k_step_partials(float* W1, float* W3, flo
 
 __global__ void k_step_apply(float* W1, float* W3, float* W2, const float* __restrict__ Dw, const float* __restrict__ Dt,
                              int H, int d, int m, float lr, int renorm, const float* __restrict__ parts) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.y;
   const int64_t n = (int64_t)m * d, n4 = n / 4;
   float4* w = reinterpret_cast<float4*>(mat_ptr(W1, W3, W2, b, H, n));

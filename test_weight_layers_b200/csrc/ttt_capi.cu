@@ -14,6 +14,7 @@
 #include <mutex>
 #include <vector>
 
+#include "kernels_nsmma.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
 #include "ttt.h"
@@ -82,7 +83,7 @@ struct Ws {
   float* XT2;          // [3H][m*d]
   float* A;            // [3H][r*r]
   float* B;            // [3H][r*r]
-  float* gram;         // [NS_GRAM_SPLIT][3H][r*r] split-K partials of the Gram matrices
+  float* gram;         // [max(NS_GRAM_SPLIT, NSM_GRAM_SPLIT_MAX)][3H][r*r] split-K partials of the Gram matrices
   float* norms;        // [3H][NORM_PARTS] partial sums of squares of G
   float* stepn;        // [3H][NORM_PARTS][2] partials of ||W||^2, ||W - lr D||^2
   float* rk;           // [T][H]
@@ -133,7 +134,7 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_XT2 = take(3 * n * 4);
   const size_t o_A = take(3 * H * r * r * 4);
   const size_t o_B = take(3 * H * r * r * 4);
-  const size_t o_gram = take((size_t)NS_GRAM_SPLIT * 3 * H * r * r * 4);
+  const size_t o_gram = take((size_t)std::max(NS_GRAM_SPLIT, NSM_GRAM_SPLIT_MAX) * 3 * H * r * r * 4);
   const size_t o_norms = take(3 * H * NORM_PARTS * 4);
   const size_t o_stepn = take(3 * H * NORM_PARTS * 2 * 4);
   const size_t o_rk = take((size_t)std::max<int64_t>(T, 1) * H * 4);
@@ -353,9 +354,31 @@ int launch_conv_any(const void* V, int64_t ldv, void* Vout, int64_t ldo, const f
   return TTT_OK;
 }
 
-int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStream_t s) {
+// Launch with programmatic stream serialisation: the kernel may begin while the
+// previous kernel on the stream finishes, and must call pdl_wait() before it
+// touches memory that kernel writes.  Used for the short dependent kernels of
+// the Muon step, whose launch latency is otherwise a large share of their time.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  TTT_CHECK(cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...));
+  return TTT_OK;
+}
+
+int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStream_t s, bool pdl = false) {
   const int64_t n = (int64_t)d.heads * d.m * d.d;
   ProfScope ps(TTT_PROF_SHADOW, s);
+  if (pdl) return launch_pdl(k_shadow, dim3(grid1d(n, 256)), dim3(256), 0, s, W.W1, W.W3, W.W2, w.wsh, w.w2b, w.wsh16,
+                             d.heads, d.d, d.m);
   k_shadow<<<grid1d(n, 256), 256, 0, s>>>(W.W1, W.W3, W.W2, w.wsh, w.w2b, w.wsh16, d.heads, d.d, d.m);
   TTT_LAUNCHED();
   return TTT_OK;
@@ -459,8 +482,70 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
 }
 
 // Newton-Schulz + weight step from G; refreshes the bf16 shadow in bf16 mode.
-int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const ttt_dims& d, const Ws& w,
-                cudaStream_t s) {
+// W <- ||W|| (W - lr D) / ||W - lr D|| with D given in W's orientation (Dw for wide, Dt for tall matrices)
+int run_step_update(const ttt_weights& W, const float* Dw, const float* Dt, const ttt_ns_cfg& ns, const ttt_dims& d,
+                    const Ws& w, cudaStream_t s) {
+  const int H = d.heads, mm = d.m, dd = d.d, nb = 3 * H;
+  const int64_t n = (int64_t)mm * dd;
+  TTT_TRY(launch_pdl(k_step_partials, dim3(nb, NORM_PARTS), dim3(256), 0, s, W.W1, W.W3, W.W2, Dw, Dt, H, dd, mm,
+                     ns.lr, w.stepn));
+  return launch_pdl(k_step_apply, dim3(grid1d(n / 4, 256) / nb + 1, nb), dim3(256), 0, s, W.W1, W.W3, W.W2, Dw, Dt, H,
+                    dd, mm, ns.lr, ns.renorm, (const float*)w.stepn);
+}
+
+// C = alpha A B + beta Cin on the tensor cores (split bf16 parts); see kernels_nsmma.cuh
+template <int NT, bool BK>
+int launch_mm3(int M, int N, int K, int ksplit, int nsplit, int batch, const float* A, int lda, int64_t sA,
+               const float* B, int ldb, int64_t sB, float* C, int ldc, int64_t sC, int64_t sCsplit, const float* Cin,
+               float alpha, float beta, const Ws& w, cudaStream_t s) {
+  auto k = k_mm3<NT, BK>;
+  TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, NsmLayout<NT>::ALLOC));
+  const dim3 grid((N + NT - 1) / NT, (M + 127) / 128, batch * nsplit);
+  return launch_pdl(k, grid, dim3(NSM_THREADS), NsmLayout<NT>::ALLOC, s, M, N, K, ksplit, nsplit, A, lda, sA, B, ldb,
+                    sB, C, ldc, sC, sCsplit, Cin, alpha, beta, w.status, wait_timeout_ns());
+}
+
+// the r x r products (Gram split-K, A A): N tile = r rounded up to 64
+template <bool BK>
+int launch_mm3_r(int r, int K, int ksplit, int nsplit, int batch, const float* A, int lda, int64_t sA, const float* B,
+                 int ldb, int64_t sB, float* C, int64_t sC, int64_t sCsplit, const float* Cin, float alpha, float beta,
+                 const Ws& w, cudaStream_t s) {
+  if (r <= 64)
+    return launch_mm3<64, BK>(r, r, K, ksplit, nsplit, batch, A, lda, sA, B, ldb, sB, C, r, sC, sCsplit, Cin, alpha,
+                              beta, w, s);
+  if (r <= 128)
+    return launch_mm3<128, BK>(r, r, K, ksplit, nsplit, batch, A, lda, sA, B, ldb, sB, C, r, sC, sCsplit, Cin, alpha,
+                               beta, w, s);
+  if (r <= 192)
+    return launch_mm3<192, BK>(r, r, K, ksplit, nsplit, batch, A, lda, sA, B, ldb, sB, C, r, sC, sCsplit, Cin, alpha,
+                               beta, w, s);
+  return TTT_ERR_UNSUPPORTED;
+}
+
+// Newton-Schulz iterations of the bf16 path on the tensor cores: X (r x c) -> X
+// after `iters` steps, then XT = X^T.  Products carry ~2^-16 relative error.
+int run_ns_iters_tc(const ttt_ns_cfg& ns, int r, int c, int nb, const Ws& w, float*& X, float*& X2, cudaStream_t s) {
+  const int64_t n = (int64_t)r * c, rr = (int64_t)r * r;
+  // Gram split-K: slices of >= 128 columns, at most NSM_GRAM_SPLIT_MAX of them
+  const int ksplit = std::max(128, ((c + NSM_GRAM_SPLIT_MAX - 1) / NSM_GRAM_SPLIT_MAX + 63) / 64 * 64);
+  const int nsplit = (c + ksplit - 1) / ksplit;
+  for (int it = 0; it < ns.iters; ++it) {
+    // Gram partials P[s][b] = X_b[:, split s] X_b[:, split s]^T (B^T rows = X rows)
+    TTT_TRY(launch_mm3_r<true>(r, c, ksplit, nsplit, nb, X, c, n, X, c, n, w.gram, rr, (int64_t)nb * rr, nullptr, 1.f,
+                               0.f, w, s));
+    TTT_TRY(launch_pdl(k_gram_reduce, dim3(grid1d((int64_t)nb * rr, 256)), dim3(256), 0, s, r, nb, nsplit,
+                       (const float*)w.gram, w.A));
+    // B = c A A + b A (A symmetric: its rows serve as B^T rows)
+    TTT_TRY(launch_mm3_r<true>(r, r, r, 1, nb, w.A, r, rr, w.A, r, rr, w.B, rr, 0, w.A, ns.c, ns.b, w, s));
+    // X' = B X + a X (B rows of X: MN-major), 128-column tiles
+    TTT_TRY((launch_mm3<128, false>(r, c, r, r, 1, nb, w.B, r, rr, X, c, n, X2, c, n, 0, X, 1.f, ns.a, w, s)));
+    std::swap(X, X2);
+  }
+  return TTT_OK;
+}
+
+int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const ttt_dims& d, ttt_dtype dt,
+                const Ws& w, cudaStream_t s) {
   const int H = d.heads, mm = d.m, dd = d.d;
   const int64_t n = (int64_t)mm * dd;
   const int nb = 3 * H;
@@ -471,9 +556,15 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
   if (ns.iters > 0) {
     k_frob_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(G, n, w.norms);
     TTT_LAUNCHED();
-    k_ns_init<<<dim3((c + 31) / 32, (c + 31) / 32, nb), dim3(32, 8), 0, s>>>(G, w.X, w.XT, w.norms, H, dd, mm, ns.eps);
-    TTT_LAUNCHED();
+    TTT_TRY(launch_pdl(k_ns_init, dim3((c + 31) / 32, (c + 31) / 32, nb), dim3(32, 8), 0, s, G, w.X, w.XT,
+                       (const float*)w.norms, H, dd, mm, ns.eps));
     float *X = w.X, *X2 = w.X2, *XT = w.XT, *XT2 = w.XT2;
+    if (dt == TTT_BF16) {
+      TTT_TRY(run_ns_iters_tc(ns, r, c, nb, w, X, X2, s));
+      TTT_TRY(launch_pdl(k_transpose_batch, dim3((c + 31) / 32, (r + 31) / 32, nb), dim3(32, 8), 0, s,
+                         (const float*)X, XT, r, c, n));
+      return run_step_update(W, X, XT, ns, d, w, s);
+    }
     const int rt = (r + 63) / 64, ct = (c + 63) / 64;
     TTT_CHECK(cudaFuncSetAttribute(k_gram_partial, cudaFuncAttributeMaxDynamicSharedMemorySize, NSC_DYN_BYTES));
     TTT_CHECK(cudaFuncSetAttribute(k_gemm_sym, cudaFuncAttributeMaxDynamicSharedMemorySize, NSC_DYN_BYTES));
@@ -482,7 +573,7 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
       // A = X X^T (from X^T), B = b A + c A A, X' = a X + B X (and X'^T)
       k_gram_partial<<<dim3(rt * (rt + 1) / 2, NS_GRAM_SPLIT, nb), 256, NSC_DYN_BYTES, s>>>(r, c, XT, n, w.gram);
       TTT_LAUNCHED();
-      k_gram_reduce<<<grid1d((int64_t)nb * rr, 256), 256, 0, s>>>(r, nb, w.gram, w.A);
+      k_gram_reduce<<<grid1d((int64_t)nb * rr, 256), 256, 0, s>>>(r, nb, NS_GRAM_SPLIT, w.gram, w.A);
       TTT_LAUNCHED();
       k_gemm_sym<<<dim3(rt, rt, nb), 256, NSC_DYN_BYTES, s>>>(r, r, w.A, rr, w.A, r, rr, w.B, r, rr, nullptr, w.A,
                                                                ns.c, ns.b);
@@ -495,18 +586,13 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
     Dw = X;
     Dt = XT;
   }
-  k_step_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(W.W1, W.W3, W.W2, Dw, Dt, H, dd, mm, ns.lr, w.stepn);
-  TTT_LAUNCHED();
-  k_step_apply<<<dim3(grid1d(n / 4, 256) / nb + 1, nb), 256, 0, s>>>(W.W1, W.W3, W.W2, Dw, Dt, H, dd, mm, ns.lr,
-                                                                    ns.renorm, w.stepn);
-  TTT_LAUNCHED();
-  return TTT_OK;
+  return run_step_update(W, Dw, Dt, ns, d, w, s);
 }
 
 int run_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const ttt_dims& d, ttt_dtype dt, const Ws& w,
              cudaStream_t s) {
-  TTT_TRY(run_ns_step(W, G, ns, d, w, s));
-  if (dt == TTT_BF16) TTT_TRY(launch_shadow(W, w, d, s));
+  TTT_TRY(run_ns_step(W, G, ns, d, dt, w, s));
+  if (dt == TTT_BF16) TTT_TRY(launch_shadow(W, w, d, s, true));
   return TTT_OK;
 }
 

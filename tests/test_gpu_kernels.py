@@ -159,7 +159,10 @@ def test_step_matches_oracle(dt, d, m, iters, renorm, lr):
                                                             Gflat[H * m * d:2 * H * m * d].reshape(H, m, d),
                                                             Gflat[2 * H * m * d:].reshape(H, d, m)))), cfg)
     errs = weight_errors(W.oracle(), ref)
-    assert max(errs) < 1e-5, errs
+    # fp32 mode: fp32 CUDA-core products.  bf16 mode: Newton-Schulz products on
+    # the tensor cores from split bf16 operands (hi + lo), ~2^-16 relative each,
+    # chained through 5 iterations of 3 products
+    assert max(errs) < (1e-5 if dt == T.TTT_FP32 else 1e-4), errs
     del dtype
 
 
