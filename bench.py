@@ -229,10 +229,11 @@ def workload_config(cfg, n, l2_note):
     return {"workload": (f"{cfg.name}: {cfg.frames} frames x ({cfg.grid_h}x{cfg.grid_w}+{cfg.special}) = "
                          f"{cfg.tokens} tokens per GPU, {cfg.heads} heads d={cfg.d} m={cfg.m}, {cfg.steps} Muon "
                          f"step(s){', ShortConv2D on V' if cfg.conv else ''}"
-                         f"{f', {cfg.n_chunks} causal chunks of {cfg.chunk}' if cfg.chunk else ''}, "
+                         f"{f', {cfg.n_chunks} causal chunks of {cfg.chunk} (' if cfg.chunk else ''}"
+                         f"{('update then apply)' if cfg.order else 'apply then update)') if cfg.chunk else ''}, "
                          f"apply on {cfg.apply_tokens} tokens"),
             "tokens_per_gpu": cfg.tokens, "heads": cfg.heads, "d": cfg.d, "m": cfg.m, "inner_steps": cfg.steps,
-            "chunk": cfg.chunk or None, "qk_l2norm": True,
+            "chunk": cfg.chunk or None, "order": cfg.order if cfg.chunk else None, "qk_l2norm": True,
             "l2": l2_note,
             "parallelism": "single GPU" if n == 1 else f"token-sharded x{n}, NCCL all-reduce of the gradient"}
 
@@ -328,7 +329,7 @@ def run_ours(args, cfg):
             T.ttt_update(Wabi, Kx, Vuse, ex, Tn, cfg.steps, ns, dm, io, ws)
             T.ttt_apply(Wabi, Qx, Ox, Ta, dm, io, ws)
         elif world == 1:
-            T.ttt_chunked(Wabi, Qx, Kx, Vuse, ex, Ox, Tn, cfg.chunk, 0, cfg.steps, ns, dm, io, ws)
+            T.ttt_chunked(Wabi, Qx, Kx, Vuse, ex, Ox, Tn, cfg.chunk, cfg.order, cfg.steps, ns, dm, io, ws)
         else:
             sharded_layer(
                 Tn, cfg.steps,
@@ -337,7 +338,7 @@ def run_ours(args, cfg):
                 step=lambda g_: T.ttt_step(Wabi, g_, ns, dm, dcode, ws),
                 apply=(lambda t0, t1: T.ttt_apply(Wabi, Qx[t0:t1], Ox[t0:t1], t1 - t0, dm, io, ws))
                 if cfg.chunk else None,
-                chunk=cfg.chunk, order=0)
+                chunk=cfg.chunk, order=cfg.order)
             if not cfg.chunk:
                 T.ttt_apply(Wabi, Qx, Ox, Ta, dm, io, ws)
 
@@ -446,7 +447,7 @@ def run_ours(args, cfg):
             def e2e_step():
                 for w, w0 in zip(W, W0):
                     w.copy_(w0, non_blocking=True)
-                T.ttt_layer_host(Wabi, hQ, hK, hV, he, hO, Tn, cfg.chunk, cfg.steps, ns, dm, io, dbuf, ws,
+                T.ttt_layer_host(Wabi, hQ, hK, hV, he, hO, Tn, cfg.chunk, cfg.order, cfg.steps, ns, dm, io, dbuf, ws,
                                  taps=taps, grid_h=cfg.grid_h if cfg.conv else 0,
                                  grid_w=cfg.grid_w if cfg.conv else 0)
             e2e_api = "ttt_layer_host (host buffers, copies overlapped with compute)"

@@ -184,9 +184,10 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
  *    being copied (block gradients are summed, so the result equals ttt_update
  *    up to the order of that sum), and each block of O is copied back as soon
  *    as it has been computed, while later queries are still arriving.
- *  - chunk > 0: the causal carry of ttt_chunked with order 0; chunk c+1 is
- *    copied in while chunk c is computed and O of chunk c is copied back
- *    meanwhile.
+ *  - chunk > 0: the causal carry of ttt_chunked with the given order (0: apply
+ *    with the carried weights, then update; 1: update, then apply); chunk c+1
+ *    is copied in while chunk c is computed and O of chunk c is copied back
+ *    meanwhile.  order must be 0 or 1 (it is not read when chunk = 0).
  *  - taps (device float [H*d][3][3]) non-null applies ShortConv2D to V over
  *    frames of grid_h x grid_w tokens first (T must be whole frames); the
  *    token blocks of chunk = 0 are then whole frames, and chunk must be too.
@@ -196,7 +197,7 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
  * streams and a pool of events per device on first use and keeps them. */
 size_t ttt_host_buffer_bytes(ttt_dims dims, int64_t T, ttt_dtype dtype, int conv);
 int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV, const float* hEta, void* hO,
-                   int64_t T, int64_t chunk, int steps, const ttt_ns_cfg* ns, const float* taps, int grid_h,
+                   int64_t T, int64_t chunk, int order, int steps, const ttt_ns_cfg* ns, const float* taps, int grid_h,
                    int grid_w, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, void* dbuf, size_t dbuf_bytes,
                    void* ws, size_t ws_bytes, void* stream);
 

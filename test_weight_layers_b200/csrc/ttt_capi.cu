@@ -940,10 +940,10 @@ size_t ttt_host_buffer_bytes(ttt_dims dims, int64_t T, ttt_dtype dtype, int conv
 }
 
 int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV, const float* hEta, void* hO,
-                   int64_t T, int64_t chunk, int steps, const ttt_ns_cfg* ns, const float* taps, int grid_h,
+                   int64_t T, int64_t chunk, int order, int steps, const ttt_ns_cfg* ns, const float* taps, int grid_h,
                    int grid_w, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, void* dbuf, size_t dbuf_bytes,
                    void* ws, size_t ws_bytes, void* stream) {
-  if (T < 0 || chunk < 0 || steps < 0) return TTT_ERR_INVALID;
+  if (T < 0 || chunk < 0 || steps < 0 || (order != 0 && order != 1)) return TTT_ERR_INVALID;
   const int64_t wsT = chunk > 0 ? std::min<int64_t>(chunk, T) : T;
   TTT_TRY(check_common(dims, dtype, wsT, ws, ws_bytes));
   TTT_TRY(check_weights(W));
@@ -1032,21 +1032,25 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
       return TTT_OK;
     };
     if (chunk > 0) {
-      // causal carry, order 0: O_c = f_(W_(c-1))(Q_c), then the update on chunk c
+      // causal carry: order 0 O_c = f_(W_(c-1))(Q_c), then the update on chunk c;
+      // order 1 the update on chunk c first, then O_c = f_(W_c)(Q_c)
       for (int64_t b = 0; b < nb; ++b) {
         const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
         TTT_CHECK(cudaStreamWaitEvent(s, ev_in[b], 0));
-        TTT_TRY(apply_block(b, w.rq));
-        if (steps == 0) continue;
-        const uint8_t* v = vsrc(t0, tb);
-        if (!v) return TTT_ERR_CUDA;
-        UpdOperands op;
-        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, dEta + t0 * dims.heads, tb, dims, dtype,
-                                        io->qk_l2norm, w, s, &op));
-        for (int st = 0; st < steps; ++st) {
-          TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s));
-          TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+        if (order == 0) TTT_TRY(apply_block(b, w.rq));
+        if (steps > 0) {
+          const uint8_t* v = vsrc(t0, tb);
+          if (!v) return TTT_ERR_CUDA;
+          UpdOperands op;
+          TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, dEta + t0 * dims.heads, tb, dims, dtype,
+                                          io->qk_l2norm, w, s, &op));
+          for (int st = 0; st < steps; ++st) {
+            TTT_TRY(
+                run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s));
+            TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+          }
         }
+        if (order == 1) TTT_TRY(apply_block(b, w.rq));
       }
       return TTT_OK;
     }

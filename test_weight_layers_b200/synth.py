@@ -24,6 +24,10 @@ Workloads (the pages give shapes, not data; these stand in for their datasets):
                 tokens, ShortConv2D on V, 2 inner steps.
 * ``loger``     LoGeR-style causal stream: 2048 frames x 32x32 = 2,097,152
                 tokens in 16 chunks of 131,072.
+* ``stream``    ZipMap streaming reconstruction: the zipmap recipe updated
+                frame by frame (chunk = one frame of 37x37 + 5 tokens, 750
+                chunks), each frame's outputs from the weights after its own
+                update (order 1).
 """
 from __future__ import annotations
 
@@ -133,6 +137,7 @@ class Workload:
     steps: int = 1
     conv: bool = False
     chunk: int = 0              # 0: one bidirectional chunk
+    order: int = 0              # chunked: 0 apply with the carried W, then update; 1 update, then apply
     query_tokens: int = 0       # >0: apply on separate query tokens instead of Q of the context
     ns_iters: int = 5
     ns_a: float = 3.4445
@@ -191,6 +196,8 @@ WORKLOADS = {
                       steps=2, conv=True),
     "loger": Workload("loger", 1004, heads=4, d=192, m=768, frames=2048, grid_h=32, grid_w=32,
                       chunk=128 * 1024),
+    "stream": Workload("stream", 1005, heads=4, d=192, m=768, frames=750, grid_h=37, grid_w=37,
+                       special=5, eta_kind="linear", chunk=37 * 37 + 5, order=1),
 }
 
 

@@ -71,7 +71,7 @@ def lib() -> ctypes.CDLL:
             "ttt_chunked": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), Dims,
                                 ctypes.POINTER(IOCfg), I, P, SZ, P]),
             "ttt_host_buffer_bytes": (SZ, [Dims, I64, I, I]),
-            "ttt_layer_host": (I, [Weights, P, P, P, P, P, I64, I64, I, ctypes.POINTER(NSCfg), P, I, I, Dims,
+            "ttt_layer_host": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), P, I, I, Dims,
                                    ctypes.POINTER(IOCfg), I, P, SZ, P, SZ, P]),
             "ttt_status_string": (ctypes.c_char_p, [I]),
             "ttt_selftest_wait_timeout": (I, [P, SZ, ctypes.c_uint, P]),
@@ -203,11 +203,12 @@ def host_buffer(dm: Dims, T: int, dtype: int, conv: bool = False, device="cuda")
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def ttt_layer_host(W: Weights, hQ, hK, hV, hEta, hO, T, chunk, steps, ns: NSCfg, dm: Dims, io: IOCfg, dbuf, ws,
-                   taps=None, grid_h=0, grid_w=0, stream=None):
+def ttt_layer_host(W: Weights, hQ, hK, hV, hEta, hO, T, chunk, order, steps, ns: NSCfg, dm: Dims, io: IOCfg, dbuf,
+                   ws, taps=None, grid_h=0, grid_w=0, stream=None):
     """hQ, hK, hV, hEta, hO are host (pinned CPU) tensors; dbuf, ws, taps and W are on the device."""
     _check("ttt_layer_host", lib().ttt_layer_host(
-        W, _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hEta), _ptr(hO), T, chunk, steps, ctypes.byref(ns), _ptr(taps), grid_h,
+        W, _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hEta), _ptr(hO), T, chunk, order, steps, ctypes.byref(ns), _ptr(taps),
+        grid_h,
         grid_w, dm, ctypes.byref(io), dtype_code(hQ.dtype), _ptr(dbuf), dbuf.numel(), _ptr(ws), ws.numel(),
         _stream(stream)))
 

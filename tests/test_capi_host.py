@@ -105,10 +105,10 @@ def test_chunked_and_conv_validation(lib):
     assert lib.ttt_shortconv2d(FAKE, 0, FAKE, 0, FAKE, 2, 4, 4, 16, 0, T.TTT_BF16, None) == T.TTT_ERR_INVALID  # alias
 
 
-def _call_layer_host(lib, dims, dtype, T_, chunk, dbuf_bytes, ws_bytes, taps=None, gh=0, gw=0, hQ=FAKE):
+def _call_layer_host(lib, dims, dtype, T_, chunk, dbuf_bytes, ws_bytes, taps=None, gh=0, gw=0, hQ=FAKE, order=0):
     W = T.Weights(1 << 20, 1 << 21, 1 << 22)
     ns, io = T.ns_cfg(), T.io_cfg()
-    return lib.ttt_layer_host(W, hQ, FAKE, FAKE, FAKE, FAKE, T_, chunk, 1, ctypes.byref(ns), taps, gh, gw, dims,
+    return lib.ttt_layer_host(W, hQ, FAKE, FAKE, FAKE, FAKE, T_, chunk, order, 1, ctypes.byref(ns), taps, gh, gw, dims,
                               ctypes.byref(io), dtype, FAKE, dbuf_bytes, FAKE, ws_bytes, None)
 
 
@@ -121,6 +121,8 @@ def test_layer_host_validation(lib):
     assert need_db >= 4 * T_ * 4 * 192 * 2 + T_ * 4 * 4
     assert T.ttt_host_buffer_bytes(d, T_, T.TTT_BF16, conv=True) >= need_db + T_ * 4 * 192 * 2
     assert T.ttt_host_buffer_bytes(T.dims(0, 192, 768), T_, T.TTT_BF16) == 0
+    assert _call_layer_host(lib, d, T.TTT_BF16, T_, 256, need_db, need_ws, order=2) == T.TTT_ERR_INVALID
+    assert _call_layer_host(lib, d, T.TTT_BF16, T_, 256, need_db, need_ws, order=-1) == T.TTT_ERR_INVALID
     assert _call_layer_host(lib, d, T.TTT_BF16, T_, 0, need_db - 1, need_ws) == T.TTT_ERR_WORKSPACE
     assert _call_layer_host(lib, d, T.TTT_BF16, T_, 0, need_db, need_ws - 1) == T.TTT_ERR_WORKSPACE
     assert _call_layer_host(lib, d, T.TTT_BF16, T_, -1, need_db, need_ws) == T.TTT_ERR_INVALID

@@ -37,7 +37,8 @@ def run_host(cfg, pinned=True):
     ws = T.workspace(dm, cfg.chunk or Tn, dt)
     dbuf = T.host_buffer(dm, Tn, dt, conv=cfg.conv)
     taps = inp.taps().cuda() if cfg.conv else None
-    T.ttt_layer_host(W.abi, hQ, hK, hV, he, hO, Tn, cfg.chunk, cfg.steps, abi_ns(cfg), dm, T.io_cfg(), dbuf, ws,
+    T.ttt_layer_host(W.abi, hQ, hK, hV, he, hO, Tn, cfg.chunk, cfg.order, cfg.steps, abi_ns(cfg), dm, T.io_cfg(),
+                     dbuf, ws,
                      taps=taps, grid_h=cfg.grid_h if cfg.conv else 0, grid_w=cfg.grid_w if cfg.conv else 0)
     check_status(ws)  # synchronises the stream: hO is complete
     return W, hO, (inp, K, V, Q, eta)
@@ -80,7 +81,7 @@ def test_host_layer_without_update_is_apply():
     hO = torch.empty((Tn, cfg.model_dim), dtype=torch.bfloat16).pin_memory()
     ws = T.workspace(dm, Tn, T.TTT_BF16)
     dbuf = T.host_buffer(dm, Tn, T.TTT_BF16)
-    T.ttt_layer_host(Wa.abi, hQ, hK, hV, he, hO, Tn, 0, 0, abi_ns(cfg), dm, T.io_cfg(), dbuf, ws)
+    T.ttt_layer_host(Wa.abi, hQ, hK, hV, he, hO, Tn, 0, 0, 0, abi_ns(cfg), dm, T.io_cfg(), dbuf, ws)
     Od = torch.empty((Tn, cfg.model_dim), dtype=torch.bfloat16, device="cuda")
     T.ttt_apply(Wa.abi, hQ.cuda(), Od, Tn, dm, T.io_cfg(), ws)
     check_status(ws)

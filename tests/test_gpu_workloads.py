@@ -1,4 +1,4 @@
-"""End-to-end GPU parity on the five workloads' recipes (update + apply through
+"""End-to-end GPU parity on the six workloads' recipes (update + apply through
 the C ABI, compared with the fp64 oracle on the same seeded inputs).
 
 The tiny (fp32) and object-scale workloads run at their full sizes; the three
@@ -46,7 +46,8 @@ def run_layer(cfg):
         T.ttt_shortconv2d(Vd, Vc, inp.taps().cuda(), cfg.frames, cfg.grid_h, cfg.grid_w, cfg.model_dim)
         Vd = Vc
     if cfg.chunk:
-        T.ttt_chunked(W.abi, Qd, Kd, Vd, ed, Od, Tn, cfg.chunk, 0, cfg.steps, abi_ns(cfg), dm, T.io_cfg(), ws)
+        T.ttt_chunked(W.abi, Qd, Kd, Vd, ed, Od, Tn, cfg.chunk, cfg.order, cfg.steps, abi_ns(cfg), dm, T.io_cfg(),
+                      ws)
     else:
         T.ttt_update(W.abi, Kd, Vd, ed, Tn, cfg.steps, abi_ns(cfg), dm, T.io_cfg(), ws)
         T.ttt_apply(W.abi, Qd, Od, Ta, dm, T.io_cfg(), ws)
@@ -58,7 +59,7 @@ def oracle_layer(cfg, inp, K, V, Q, eta):
     W0 = O.FastWeights.of(*(w.numpy() for w in inp.weights()))
     conv = (inp.taps().double().numpy(), cfg.frames, cfg.grid_h, cfg.grid_w, 0) if cfg.conv else None
     if cfg.chunk:
-        return O.chunked(W0, f64(Q), f64(K), f64(V), f64(eta), cfg.chunk, cfg.steps, ns_of(cfg), order=0)
+        return O.chunked(W0, f64(Q), f64(K), f64(V), f64(eta), cfg.chunk, cfg.steps, ns_of(cfg), order=cfg.order)
     Wf = O.update(W0, f64(K), f64(V), f64(eta), cfg.steps, ns_of(cfg), conv=conv)
     return Wf, O.apply(Wf, f64(Q))
 
@@ -69,6 +70,7 @@ CASES = {
     "zipmap-12f": S.WORKLOADS["zipmap"].with_frames(12),
     "vggt3-4f": S.WORKLOADS["vggt3"].with_frames(4),
     "loger-16f": S.WORKLOADS["loger"].with_frames(16, chunk=4096),
+    "stream-6f": S.WORKLOADS["stream"].with_frames(6),
 }
 
 
