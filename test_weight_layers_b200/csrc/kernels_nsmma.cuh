@@ -261,3 +261,480 @@ __global__ void k_transpose_batch(const float* __restrict__ X, float* __restrict
 }
 
 }  // namespace ttt
+
+namespace ttt {
+
+// ---------------------------------------------------------------------------
+// The whole Newton-Schulz loop of one matrix in one launch (bf16 mode).
+//
+// A cluster of CS = c / 128 CTAs per matrix; CTA j owns columns
+// [128 j, 128 j + 128) of the wide iterate X (R x c, R in {128, 192}), which is
+// updated in place in global memory.  With A = X X^T kept in global memory
+// (R x R), one iteration is, in every CTA:
+//   1. B = cc A A^T + b A, computed whole by each CTA (K = R, both operands are
+//      A's rows, resident in shared memory; A is symmetric up to rounding);
+//   2. X_j <- B X_j + a X_j for its own columns (K = R in 64-row chunks through
+//      two staging buffers);
+//   3. unless it is the last iteration: P_j = X_j X_j^T (K = 128) into an fp32
+//      shared tile; cluster barrier; CTA j sums the rows i = j (mod CS) of
+//      A = sum_q P_q over q = 0..CS-1 in that fixed order, reading the other
+//      CTAs' tiles through distributed shared memory, and writes them; cluster
+//      barrier.
+// Step 3 also runs once on X_0 before the first iteration.  Products use split
+// bf16 operands (hi*hi + hi*lo + lo*hi, fp32 accumulation in TMEM) as in k_mm3.
+// M tiles of 128 rows: rows 0..127 and, for R = 192, rows 64..191 (of the second
+// tile only rows 128..191 are kept).  All threads stage operands; one elected
+// thread issues the MMAs; every CTA runs the same sequence of cluster barriers
+// whatever happens, so a failed wait (recorded in the status word) never
+// leaves a peer waiting at a barrier.
+
+constexpr int NSC_THREADS = 256;
+constexpr int NSC_COLS = 128;  // columns of X per CTA
+
+template <int R>
+struct NscLayout {
+  static constexpr int KB = R / 64;                          // 64-wide K blocks of an R-wide operand
+  static constexpr int ROWBLK = R * 128;                     // one [R rows][64 bf16] K block, 128-byte swizzle
+  static constexpr int PART = KB * ROWBLK;                   // one bf16 part (hi or lo) of an R x R operand
+  static constexpr int P_LD = R + 4;                         // fp32 P tile row stride (floats)
+  static constexpr int OPS = 2 * PART > R * P_LD * 4 ? 2 * PART : R * P_LD * 4;
+  static constexpr int OPA_BYTES = (OPS + 1023) / 1024 * 1024;
+  static constexpr int XCH = 64 * NSC_COLS * 2;              // one part of an X chunk: 2 MN blocks [64 k][64 n]
+  static constexpr int XSTAGE = 2 * XCH;                     // hi + lo
+  static constexpr int XST_OFF = OPA_BYTES;
+  static constexpr int BAR_OFF = XST_OFF + 2 * XSTAGE;
+  static constexpr int ALLOC = BAR_OFF + 64 + 1024;
+  static constexpr int NMT = R == 192 ? 2 : 1;               // M tiles
+  static_assert(8 * 32 * 36 * 4 <= 2 * XSTAGE, "transpose buffers fit the X stages");
+  static_assert(R == 128 || R == 192, "rows");
+  static_assert(ALLOC <= 232448, "shared memory budget");
+  static_assert(NMT * R <= 512, "TMEM budget");
+};
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// 32 consecutive fp32 values (one row, from registers) -> bf16 hi/lo parts of a
+// K-major operand: columns col0..col0+31 of row `row` (col0 a multiple of 32)
+template <int ROWBLK, int PART>
+__device__ __forceinline__ void nsc_put_row32(uint8_t* op, int row, int col0, const float* x) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int col = col0 + 8 * c;
+    uint4 hi, lo;
+    nsm_split8(make_float4(x[8 * c], x[8 * c + 1], x[8 * c + 2], x[8 * c + 3]),
+               make_float4(x[8 * c + 4], x[8 * c + 5], x[8 * c + 6], x[8 * c + 7]), hi, lo);
+    const uint32_t off = (col >> 6) * ROWBLK + sw128_offset(row, (col & 63) >> 3);
+    *reinterpret_cast<uint4*>(op + off) = hi;
+    *reinterpret_cast<uint4*>(op + PART + off) = lo;
+  }
+}
+
+// 8 floats through L2 (data written by other CTAs of the cluster in this kernel)
+__device__ __forceinline__ void nsc_load8_cg(const float* p, float4& u, float4& v) {
+  u = __ldcg(reinterpret_cast<const float4*>(p));
+  v = __ldcg(reinterpret_cast<const float4*>(p + 4));
+}
+
+// inverse of nsc_put_row32: hi + lo of columns col0..col0+31 of row `row`
+template <int ROWBLK, int PART>
+__device__ __forceinline__ void nsc_get_row32(const uint8_t* op, int row, int col0, float* x) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int col = col0 + 8 * c;
+    const uint32_t off = (col >> 6) * ROWBLK + sw128_offset(row, (col & 63) >> 3);
+    const uint4 hi = *reinterpret_cast<const uint4*>(op + off);
+    const uint4 lo = *reinterpret_cast<const uint4*>(op + PART + off);
+    const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w}, lw[4] = {lo.x, lo.y, lo.z, lo.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 h2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[e]));
+      const float2 l2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[e]));
+      x[8 * c + 2 * e] = h2.x + l2.x;
+      x[8 * c + 2 * e + 1] = h2.y + l2.y;
+    }
+  }
+}
+
+template <int R>
+__global__ void __launch_bounds__(NSC_THREADS, 1)
+    k_ns_cluster(float* X, float* A, int c, int iters, float na, float nb_, float nc,
+                 unsigned int* status, unsigned long long timeout_ns) {
+  using L = NscLayout<R>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* opa = smem;                   // K-major operands (hi part, then lo part) / fp32 P tile
+  uint8_t* xst = smem + L::XST_OFF;      // [2] X chunk stages (MN-major, hi then lo)
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);  // MMAs of a phase complete
+  uint64_t* xbar = mbar + 1;                                        // [2] MMAs of an X stage complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 2);
+  float* ptile = reinterpret_cast<float*>(opa);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int CS = (int)gridDim.x;  // cluster = the CTAs of one matrix
+  const int j = (int)cluster_ctarank();
+  const int b = blockIdx.y;
+  X += (int64_t)b * R * c;
+  A += (int64_t)b * R * R;
+  const int col_base = j * NSC_COLS;
+  pdl_trigger();
+
+  if (tid == 0) {
+    mbar_init(mbar, 1);
+    mbar_init(xbar, 1);
+    mbar_init(xbar + 1, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // X comes from the previous kernel on the stream
+  const Guard g{status, timeout_ns};
+  bool ok = true;
+  uint32_t mph = 0, xph0 = 0, xph1 = 0;
+  const bool issuer = warp == 0;
+  const uint64_t d_oh = sdesc_sw128(smem_u32(opa), 16, 1024);
+  const uint64_t d_ol = sdesc_sw128(smem_u32(opa + L::PART), 16, 1024);
+  constexpr uint32_t ID_RR = idesc_bf16(128, R, false, false);         // B = A A^T, P = X X^T
+  constexpr uint32_t ID_BX = idesc_bf16(128, NSC_COLS, false, true);   // B X (X chunk MN-major)
+  const int q = warp & 3, half = warp >> 2;
+  const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+
+  // wait for the MMAs committed to `bar` (all threads; uniform result)
+  auto wait_bar = [&](uint64_t* bar, uint32_t& ph) {
+    const bool w = ok ? mbar_wait(bar, ph, g) : false;
+    ph ^= 1u;
+    ok = __syncthreads_and(w ? 1 : 0) != 0 && ok;
+    tc_fence_after();
+  };
+  // three MMAs of one split product k step
+  auto mma3 = [&](uint32_t d, uint64_t ah, uint64_t al, uint64_t bh, uint64_t bl, uint32_t id, uint32_t acc) {
+    umma_bf16_ss(d, ah, bh, id, acc);
+    umma_bf16_ss(d, ah, bl, id, 1u);
+    umma_bf16_ss(d, al, bh, id, 1u);
+  };
+  // rows of M tile t held by TMEM lane quarter q: tile 0 all, tile 1 (R = 192) quarters 2, 3 (rows 128..191)
+  auto tile_row = [&](int t) { return t == 0 ? q * 32 + lane : 64 + q * 32 + lane; };
+  auto tile_has = [&](int t) { return t == 0 || q >= 2; };
+
+  // Gram of the CTA's columns from the operand in `opa` (K-major [R][128]) into
+  // the fp32 tile, then the cluster reduction of A's rows
+  auto gram_and_reduce = [&]() {
+    fence_async_smem();
+    __syncthreads();
+    if (ok && issuer) {
+      tc_fence_after();
+      if (elect_one()) {
+#pragma unroll
+        for (int t = 0; t < L::NMT; ++t)
+#pragma unroll
+          for (int kb = 0; kb < NSC_COLS / 64; ++kb)
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+              const uint32_t ao = (uint32_t)(kb * L::ROWBLK + t * 64 * 128 + s * 32) >> 4;
+              const uint32_t bo = (uint32_t)(kb * L::ROWBLK + s * 32) >> 4;
+              mma3(tmem + t * R, d_oh + ao, d_ol + ao, d_oh + bo, d_ol + bo, ID_RR, (kb | s) ? 1u : 0u);
+            }
+        umma_commit(mbar);
+      }
+      __syncwarp();
+    }
+    wait_bar(mbar, mph);
+    // TMEM -> fp32 tile [R][P_LD] (the operands are no longer needed)
+#pragma unroll
+    for (int t = 0; t < L::NMT; ++t) {
+      if (!tile_has(t)) continue;
+      const int row = tile_row(t);
+      for (int c0 = half * (R / 2); c0 < (half + 1) * (R / 2); c0 += 32) {
+        uint32_t v[32];
+        if (ok) {
+          tmem_ld32(tmem + lane_base + t * R + c0, v);
+          tmem_ld_wait(v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        float* dst = ptile + row * L::P_LD + c0;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+      }
+    }
+    tc_fence_before();
+    cluster_sync_all();  // every CTA's P tile is complete
+    // rows i = j (mod CS): A[i][:] = sum_q P_q[i][:], q in order
+    {
+      // three items per thread at a time, the CS partial tiles of all in flight at once
+      constexpr int V4 = R / 4;
+      const int nrows = (R - j + CS - 1) / CS;
+      const int items = nrows * V4;
+      for (int idx0 = tid; idx0 < items; idx0 += 3 * NSC_THREADS) {
+        float4 pv[3][8];
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+          const int idx = idx0 + u * NSC_THREADS;
+          const int i = j + (idx / V4) * CS, c4 = idx % V4;
+          const float* src = ptile + (idx < items ? i * L::P_LD + c4 * 4 : 0);
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq)
+            if (qq < CS) pv[u][qq] = ld_cluster_f4(cluster_addr(src, (uint32_t)qq));
+        }
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+          const int idx = idx0 + u * NSC_THREADS;
+          if (idx >= items) continue;
+          float4 acc = pv[u][0];
+#pragma unroll
+          for (int qq = 1; qq < 8; ++qq)
+            if (qq < CS) {
+              acc.x += pv[u][qq].x;
+              acc.y += pv[u][qq].y;
+              acc.z += pv[u][qq].z;
+              acc.w += pv[u][qq].w;
+            }
+          const int i = j + (idx / V4) * CS, c4 = idx % V4;
+          *reinterpret_cast<float4*>(A + (int64_t)i * R + c4 * 4) = acc;
+        }
+      }
+    }
+    cluster_sync_all();  // A complete (global writes released to the cluster), peers done with the tiles
+    tc_fence_after();
+  };
+
+  // ---- X_0: Gram operand from global (rows 0..R-1, the CTA's 128 columns)
+  {
+    constexpr int ITEMS = R * (NSC_COLS / 8), BATCH = (ITEMS / NSC_THREADS) % 6 == 0 ? 6 : 4;
+    static_assert(ITEMS % (NSC_THREADS * BATCH) == 0, "staging batches");
+    for (int i0 = 0; i0 < ITEMS / NSC_THREADS; i0 += BATCH) {
+      float4 u[BATCH], v[BATCH];
+#pragma unroll
+      for (int i = 0; i < BATCH; ++i) {
+        const int idx = tid + (i0 + i) * NSC_THREADS, row = idx >> 4, c8 = idx & 15;
+        nsm_load8(X + (int64_t)row * c + col_base + c8 * 8, true, u[i], v[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < BATCH; ++i) {
+        const int idx = tid + (i0 + i) * NSC_THREADS, row = idx >> 4, c8 = idx & 15;
+        uint4 hi, lo;
+        nsm_split8(u[i], v[i], hi, lo);
+        const uint32_t off = (c8 >> 3) * L::ROWBLK + sw128_offset(row, c8 & 7);
+        *reinterpret_cast<uint4*>(opa + off) = hi;
+        *reinterpret_cast<uint4*>(opa + L::PART + off) = lo;
+      }
+    }
+  }
+  gram_and_reduce();
+
+  for (int it = 0; it < iters; ++it) {
+    const bool last = it + 1 == iters;
+    // ---- 1. B = nc A A^T + nb A
+    {
+      constexpr int ITEMS = R * (R / 8), BATCH = (ITEMS / NSC_THREADS) % 9 == 0 ? 9 : 8;
+      static_assert(ITEMS % (NSC_THREADS * BATCH) == 0, "staging batches");
+      for (int i0 = 0; i0 < ITEMS / NSC_THREADS; i0 += BATCH) {
+        float4 u[BATCH], v[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int idx = tid + (i0 + i) * NSC_THREADS, row = idx / (R / 8), c8 = idx % (R / 8);
+          nsc_load8_cg(A + (int64_t)row * R + c8 * 8, u[i], v[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int idx = tid + (i0 + i) * NSC_THREADS, row = idx / (R / 8), c8 = idx % (R / 8);
+          uint4 hi, lo;
+          nsm_split8(u[i], v[i], hi, lo);
+          const uint32_t off = (c8 >> 3) * L::ROWBLK + sw128_offset(row, c8 & 7);
+          *reinterpret_cast<uint4*>(opa + off) = hi;
+          *reinterpret_cast<uint4*>(opa + L::PART + off) = lo;
+        }
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (ok && issuer) {
+      tc_fence_after();
+      if (elect_one()) {
+#pragma unroll
+        for (int t = 0; t < L::NMT; ++t)
+#pragma unroll
+          for (int kb = 0; kb < L::KB; ++kb)
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+              const uint32_t ao = (uint32_t)(kb * L::ROWBLK + t * 64 * 128 + s * 32) >> 4;
+              const uint32_t bo = (uint32_t)(kb * L::ROWBLK + s * 32) >> 4;
+              mma3(tmem + t * R, d_oh + ao, d_ol + ao, d_oh + bo, d_ol + bo, ID_RR, (kb | s) ? 1u : 0u);
+            }
+        umma_commit(mbar);
+      }
+      __syncwarp();
+    }
+    wait_bar(mbar, mph);
+    // B rows -> K-major operand in place of A's.  The b A term takes A = hi + lo
+    // (within 2^-17 relative) from the operand itself: each thread reads exactly
+    // the entries it then overwrites.
+#pragma unroll
+    for (int t = 0; t < L::NMT; ++t) {
+      if (!tile_has(t)) continue;
+      const int row = tile_row(t);
+      for (int c0 = half * (R / 2); c0 < (half + 1) * (R / 2); c0 += 32) {
+        float x[32];
+        nsc_get_row32<L::ROWBLK, L::PART>(opa, row, c0, x);
+        uint32_t v[32];
+        if (ok) {
+          tmem_ld32(tmem + lane_base + t * R + c0, v);
+          tmem_ld_wait(v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = fmaf(nb_, x[e], nc * __uint_as_float(v[e]));
+        nsc_put_row32<L::ROWBLK, L::PART>(opa, row, c0, x);
+      }
+    }
+    tc_fence_before();
+    fence_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    // ---- 2. X_j <- B X_j + a X_j: X rows in 64-row chunks (MN-major [64 k][128 n]) through two stages
+    for (int kc = 0; kc < L::KB; ++kc) {
+      const int st = kc & 1;
+      uint8_t* xs = xst + st * L::XSTAGE;
+      if (kc >= 2) wait_bar(xbar + st, st ? xph1 : xph0);  // chunk kc - 2's MMAs released the stage
+      {
+        constexpr int ITEMS = 64 * (NSC_COLS / 8), IT = ITEMS / NSC_THREADS;
+        float4 u[IT], v[IT];
+#pragma unroll
+        for (int i = 0; i < IT; ++i) {
+          const int idx = tid + i * NSC_THREADS, kr = idx >> 4, c8 = idx & 15;
+          nsm_load8(X + (int64_t)(kc * 64 + kr) * c + col_base + c8 * 8, true, u[i], v[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < IT; ++i) {
+          const int idx = tid + i * NSC_THREADS, kr = idx >> 4, c8 = idx & 15;
+          uint4 hi, lo;
+          nsm_split8(u[i], v[i], hi, lo);
+          const uint32_t off = (c8 >> 3) * (64 * 128) + sw128_offset(kr, c8 & 7);
+          *reinterpret_cast<uint4*>(xs + off) = hi;
+          *reinterpret_cast<uint4*>(xs + L::XCH + off) = lo;
+        }
+      }
+      fence_async_smem();
+      __syncthreads();
+      if (ok && issuer) {
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t d_xh = sdesc_sw128(smem_u32(xs), 64 * 128, 1024);
+          const uint64_t d_xl = sdesc_sw128(smem_u32(xs + L::XCH), 64 * 128, 1024);
+#pragma unroll
+          for (int t = 0; t < L::NMT; ++t)
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+              const uint32_t ao = (uint32_t)(kc * L::ROWBLK + t * 64 * 128 + s * 32) >> 4;
+              const uint32_t bo = (uint32_t)(s * 2048) >> 4;
+              mma3(tmem + t * NSC_COLS, d_oh + ao, d_ol + ao, d_xh + bo, d_xl + bo, ID_BX, (kc | s) ? 1u : 0u);
+            }
+          umma_commit(xbar + st);
+        }
+        __syncwarp();
+      }
+    }
+    // X values of the tile-0 row of this thread (the a X term), loaded while the MMAs finish
+    float xpre[64];
+    {
+      const float4* xr = reinterpret_cast<const float4*>(X + (int64_t)tile_row(0) * c + col_base + half * 64);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float4 a4 = xr[e];
+        xpre[4 * e] = a4.x;
+        xpre[4 * e + 1] = a4.y;
+        xpre[4 * e + 2] = a4.z;
+        xpre[4 * e + 3] = a4.w;
+      }
+    }
+    // the last chunk's commit covers every MMA of the product
+    {
+      const int st = (L::KB - 1) & 1;
+      wait_bar(xbar + st, st ? xph1 : xph0);
+      // the other stage's last commit is complete too; keep its phase in step
+      if (L::KB >= 2) {
+        if (st) xph0 ^= 1u;
+        else xph1 ^= 1u;
+      }
+    }
+    // X' = acc + a X -> global (in place) and, unless last, the Gram operand
+    float* tbuf = reinterpret_cast<float*>(xst) + warp * (32 * 36);
+#pragma unroll
+    for (int t = 0; t < L::NMT; ++t) {
+      if (!tile_has(t)) continue;
+      const int row = tile_row(t);
+      float* xr = X + (int64_t)row * c + col_base;
+      if (t > 0) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float4 a4 = reinterpret_cast<const float4*>(xr + half * 64)[e];
+          xpre[4 * e] = a4.x;
+          xpre[4 * e + 1] = a4.y;
+          xpre[4 * e + 2] = a4.z;
+          xpre[4 * e + 3] = a4.w;
+        }
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int c0 = half * 64 + h2 * 32;
+        float x[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = xpre[h2 * 32 + e];
+        uint32_t v[32];
+        if (ok) {
+          tmem_ld32(tmem + lane_base + t * NSC_COLS + c0, v);
+          tmem_ld_wait(v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = fmaf(na, x[e], __uint_as_float(v[e]));
+        // X' rows leave through the warp's 32 x 32 transpose buffer (row stride 36
+        // floats: conflict-free both ways), so that each store writes 4 whole
+        // 128-byte row segments instead of 32 scattered 16-byte pieces
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(tbuf + lane * 36 + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+        __syncwarp();
+        {
+          const int rbase = row - lane;  // first row of this warp's 32
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rr = 4 * k + (lane >> 3), cc = (lane & 7) * 4;
+            *reinterpret_cast<float4*>(X + (int64_t)(rbase + rr) * c + col_base + c0 + cc) =
+                *reinterpret_cast<const float4*>(tbuf + rr * 36 + cc);
+          }
+        }
+        if (!last) nsc_put_row32<L::ROWBLK, L::PART>(opa, row, c0, x);
+      }
+    }
+    tc_fence_before();
+    if (!last) gram_and_reduce();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace ttt

@@ -544,6 +544,55 @@ int run_ns_iters_tc(const ttt_ns_cfg& ns, int r, int c, int nb, const Ws& w, flo
   return TTT_OK;
 }
 
+// One launch for all Newton-Schulz iterations of the bf16 path: a cluster of
+// c / 128 CTAs per matrix (k_ns_cluster), X updated in place.  Usable when
+// r is 128 or 192, c is a multiple of 128 with at most 8 column blocks, and
+// such a cluster fits on the device.
+template <int R>
+int ns_cluster_launch(int c, int nb, const ttt_ns_cfg& ns, const Ws& w, cudaStream_t s, bool probe_only,
+                      bool* fits) {
+  auto k = k_ns_cluster<R>;
+  TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, NscLayout<R>::ALLOC));
+  const int cs = c / NSC_COLS;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, nb);
+  cfg.blockDim = dim3(NSC_THREADS);
+  cfg.dynamicSmemBytes = NscLayout<R>::ALLOC;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  if (probe_only) {
+    int n = 0;
+    cfg.numAttrs = 1;
+    *fits = cudaOccupancyMaxActiveClusters(&n, k, &cfg) == cudaSuccess && n >= 1;
+    (void)cudaGetLastError();
+    return TTT_OK;
+  }
+  TTT_CHECK(cudaLaunchKernelEx(&cfg, k, w.X, w.A, c, ns.iters, ns.a, ns.b, ns.c, w.status, wait_timeout_ns()));
+  return TTT_OK;
+}
+
+bool ns_cluster_usable(int r, int c) {
+  if ((r != 128 && r != 192) || c % NSC_COLS || c / NSC_COLS < 1 || c / NSC_COLS > 8) return false;
+  static std::atomic<int> cache[2][9] = {};  // 0 unknown, 1 fits, 2 does not
+  std::atomic<int>& e = cache[r == 192][c / NSC_COLS];
+  if (e.load() == 0) {
+    bool fits = false;
+    const Ws none{};
+    const int rc = r == 192 ? ns_cluster_launch<192>(c, 1, ttt_ns_cfg{}, none, nullptr, true, &fits)
+                            : ns_cluster_launch<128>(c, 1, ttt_ns_cfg{}, none, nullptr, true, &fits);
+    e.store(rc == TTT_OK && fits ? 1 : 2);
+  }
+  return e.load() == 1;
+}
+
 int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const ttt_dims& d, ttt_dtype dt,
                 const Ws& w, cudaStream_t s) {
   const int H = d.heads, mm = d.m, dd = d.d;
@@ -560,7 +609,13 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
                        (const float*)w.norms, H, dd, mm, ns.eps));
     float *X = w.X, *X2 = w.X2, *XT = w.XT, *XT2 = w.XT2;
     if (dt == TTT_BF16) {
-      TTT_TRY(run_ns_iters_tc(ns, r, c, nb, w, X, X2, s));
+      if (ns_cluster_usable(r, c)) {
+        bool unused = false;
+        TTT_TRY(r == 192 ? ns_cluster_launch<192>(c, nb, ns, w, s, false, &unused)
+                         : ns_cluster_launch<128>(c, nb, ns, w, s, false, &unused));
+      } else {
+        TTT_TRY(run_ns_iters_tc(ns, r, c, nb, w, X, X2, s));
+      }
       TTT_TRY(launch_pdl(k_transpose_batch, dim3((c + 31) / 32, (r + 31) / 32, nb), dim3(32, 8), 0, s,
                          (const float*)X, XT, r, c, n));
       return run_step_update(W, X, XT, ns, d, w, s);
