@@ -638,7 +638,6 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     bool ok = true;
     for (int item = pair; ok && item < n_items; item += npairs, ++it) {
       const int tile = item / H, h = item % H;
-      const int64_t t = (int64_t)tile * 2 * TC_TILE + (int64_t)rank * TC_TILE + row;
       float r = 1.f;
       for (int c = 0; c < nc; ++c, ++gc) {
         const int hb = gc & 1;
