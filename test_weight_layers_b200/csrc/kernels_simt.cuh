@@ -491,27 +491,57 @@ __global__ void __launch_bounds__(256, 2) k_shortconv_band(const T* __restrict__
 //   Wsh (bf16, apply) and Wsh16 (fp16, gradient) rows [0, Hm): W1 [H][m][d];
 //   [Hm, 2Hm): W3;  [2Hm, 3Hm): W2^T [H][m][d];   W2b [H][d][m] (bf16 W2, apply)
 
-__global__ void k_shadow(const float* __restrict__ W1, const float* __restrict__ W3, const float* __restrict__ W2,
-                         __nv_bfloat16* __restrict__ Wsh, __nv_bfloat16* __restrict__ W2b, __half* __restrict__ Wsh16,
-                         int H, int d, int m) {
+// Blocks [0, n/1024): the element-wise copies, four elements per thread (16-byte
+// reads, 8-byte writes).  Blocks past that: W2^T in 32 x 32 tiles through
+// shared memory, so both the W2 reads and the W2^T writes are row-contiguous.
+// n = H*m*d is a multiple of 1024 (m a multiple of 64, d of 16).
+constexpr int SHADOW_EW_BLOCK = 256 * 4;
+
+__device__ __forceinline__ uint2 pack4_bf16(float4 v) {
+  return make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+}
+__device__ __forceinline__ uint2 pack4_f16(float4 v) {
+  return make_uint2(pack_f16x2(v.x, v.y), pack_f16x2(v.z, v.w));
+}
+
+__global__ void __launch_bounds__(256) k_shadow(const float* __restrict__ W1, const float* __restrict__ W3,
+                                                const float* __restrict__ W2, __nv_bfloat16* __restrict__ Wsh,
+                                                __nv_bfloat16* __restrict__ W2b, __half* __restrict__ Wsh16, int H,
+                                                int d, int m) {
   pdl_trigger();
   pdl_wait();
   const int64_t n = (int64_t)H * m * d;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    Wsh[i] = __float2bfloat16_rn(W1[i]);
-    Wsh[n + i] = __float2bfloat16_rn(W3[i]);
-    // i indexes W2^T [h][j][k]  <-  W2 [h][k][j]
-    const int64_t h = i / ((int64_t)m * d);
-    const int64_t rem = i % ((int64_t)m * d);
-    const int64_t j = rem / d, k = rem % d;
-    const float w2t = W2[(h * d + k) * m + j];
-    Wsh[2 * n + i] = __float2bfloat16_rn(w2t);
-    W2b[i] = __float2bfloat16_rn(W2[i]);
+  const int ew_blocks = (int)(n / SHADOW_EW_BLOCK);
+  if ((int)blockIdx.x < ew_blocks) {
+    const int64_t i = ((int64_t)blockIdx.x * 256 + threadIdx.x) * 4;
+    const float4 a = *reinterpret_cast<const float4*>(W1 + i);
+    const float4 b = *reinterpret_cast<const float4*>(W3 + i);
+    const float4 c = *reinterpret_cast<const float4*>(W2 + i);
+    *reinterpret_cast<uint2*>(Wsh + i) = pack4_bf16(a);
+    *reinterpret_cast<uint2*>(Wsh + n + i) = pack4_bf16(b);
+    *reinterpret_cast<uint2*>(W2b + i) = pack4_bf16(c);
     if (Wsh16) {  // fp16 copy only when a gradient kernel will read it
-      Wsh16[i] = __float2half_rn(W1[i]);
-      Wsh16[n + i] = __float2half_rn(W3[i]);
-      Wsh16[2 * n + i] = __float2half_rn(w2t);
+      *reinterpret_cast<uint2*>(Wsh16 + i) = pack4_f16(a);
+      *reinterpret_cast<uint2*>(Wsh16 + n + i) = pack4_f16(b);
     }
+    return;
+  }
+  // W2^T [h][j][k] <- W2 [h][k][j]: tile (h, k0, j0) of 32 x 32
+  __shared__ float tile[32][33];
+  const int t = (int)blockIdx.x - ew_blocks;
+  const int kt = d / 32, jt = m / 32;
+  const int h = t / (kt * jt), rem = t % (kt * jt);
+  const int k0 = (rem / jt) * 32, j0 = (rem % jt) * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  const float* src = W2 + (int64_t)h * d * m;
+  for (int y = ty; y < 32; y += 8) tile[y][tx] = src[(int64_t)(k0 + y) * m + j0 + tx];
+  __syncthreads();
+  const int64_t base = 2 * n + (int64_t)h * m * d;
+  for (int y = ty; y < 32; y += 8) {
+    const float v = tile[tx][y];  // W2[k0 + tx][j0 + y]
+    const int64_t o = base + (int64_t)(j0 + y) * d + k0 + tx;
+    Wsh[o] = __float2bfloat16_rn(v);
+    if (Wsh16) Wsh16[o] = __float2half_rn(v);
   }
 }
 

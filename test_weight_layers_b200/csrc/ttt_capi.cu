@@ -376,10 +376,13 @@ int launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStre
 
 int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStream_t s, bool pdl = false) {
   const int64_t n = (int64_t)d.heads * d.m * d.d;
+  if (n % SHADOW_EW_BLOCK || d.d % 32 || d.m % 32) return TTT_ERR_UNSUPPORTED;
+  const int blocks = (int)(n / SHADOW_EW_BLOCK) + d.heads * (d.d / 32) * (d.m / 32);
   ProfScope ps(TTT_PROF_SHADOW, s);
-  if (pdl) return launch_pdl(k_shadow, dim3(grid1d(n, 256)), dim3(256), 0, s, W.W1, W.W3, W.W2, w.wsh, w.w2b, w.wsh16,
-                             d.heads, d.d, d.m);
-  k_shadow<<<grid1d(n, 256), 256, 0, s>>>(W.W1, W.W3, W.W2, w.wsh, w.w2b, w.wsh16, d.heads, d.d, d.m);
+  if (pdl)
+    return launch_pdl(k_shadow, dim3(blocks), dim3(256), 0, s, W.W1, W.W3, W.W2, w.wsh, w.w2b, w.wsh16, d.heads, d.d,
+                      d.m);
+  k_shadow<<<blocks, 256, 0, s>>>(W.W1, W.W3, W.W2, w.wsh, w.w2b, w.wsh16, d.heads, d.d, d.m);
   TTT_LAUNCHED();
   return TTT_OK;
 }

@@ -138,9 +138,13 @@ def test_grad_is_deterministic(dt):
     assert torch.equal(G1, G2)
 
 
-@pytest.mark.parametrize("dt,d,m", [(T.TTT_BF16, 192, 768), (T.TTT_BF16, 128, 64), (T.TTT_FP32, 64, 128),
-                                    (T.TTT_FP32, 96, 32)])
-@pytest.mark.parametrize("iters,renorm,lr", [(5, 1, 1.0), (0, 0, 0.01), (3, 0, 0.5)])
+# bf16 shapes cover every Newton-Schulz path: one cluster launch with 192 rows and
+# 6 or 3 column blocks, with 128 rows and 2 or 1 blocks; per-product launches
+# for 192 x 320 (columns not a multiple of 128) and 64 x 128 (64 rows)
+@pytest.mark.parametrize("dt,d,m", [(T.TTT_BF16, 192, 768), (T.TTT_BF16, 192, 384), (T.TTT_BF16, 128, 256),
+                                    (T.TTT_BF16, 128, 128), (T.TTT_BF16, 192, 320), (T.TTT_BF16, 128, 64),
+                                    (T.TTT_FP32, 64, 128), (T.TTT_FP32, 96, 32)])
+@pytest.mark.parametrize("iters,renorm,lr", [(5, 1, 1.0), (0, 0, 0.01), (3, 0, 0.5), (1, 1, 1.0)])
 def test_step_matches_oracle(dt, d, m, iters, renorm, lr):
     H = 2
     W = DevWeights(*rand_weights(H, d, m, 40))
