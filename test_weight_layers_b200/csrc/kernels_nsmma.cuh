@@ -475,14 +475,14 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
     cluster_sync_all();  // every CTA's P tile is complete
     // rows i = j (mod CS): A[i][:] = sum_q P_q[i][:], q in order
     {
-      // three items per thread at a time, the CS partial tiles of all in flight at once
+      // two items per thread at a time, the CS partial tiles of both in flight at once
       constexpr int V4 = R / 4;
       const int nrows = (R - j + CS - 1) / CS;
       const int items = nrows * V4;
-      for (int idx0 = tid; idx0 < items; idx0 += 3 * NSC_THREADS) {
-        float4 pv[3][8];
+      for (int idx0 = tid; idx0 < items; idx0 += 2 * NSC_THREADS) {
+        float4 pv[2][8];
 #pragma unroll
-        for (int u = 0; u < 3; ++u) {
+        for (int u = 0; u < 2; ++u) {
           const int idx = idx0 + u * NSC_THREADS;
           const int i = j + (idx / V4) * CS, c4 = idx % V4;
           const float* src = ptile + (idx < items ? i * L::P_LD + c4 * 4 : 0);
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
             if (qq < CS) pv[u][qq] = ld_cluster_f4(cluster_addr(src, (uint32_t)qq));
         }
 #pragma unroll
-        for (int u = 0; u < 3; ++u) {
+        for (int u = 0; u < 2; ++u) {
           const int idx = idx0 + u * NSC_THREADS;
           if (idx >= items) continue;
           float4 acc = pv[u][0];
@@ -510,6 +510,27 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
     }
     cluster_sync_all();  // A complete (global writes released to the cluster), peers done with the tiles
     tc_fence_after();
+  };
+
+  // X rows [64 kc, 64 kc + 64) of the CTA's columns -> stage st (MN-major [64 k][128 n], hi then lo)
+  auto stage_x = [&](int kc, int st) {
+    uint8_t* xs = xst + st * L::XSTAGE;
+    constexpr int ITEMS = 64 * (NSC_COLS / 8), IT = ITEMS / NSC_THREADS;
+    float4 u[IT], v[IT];
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+      const int idx = tid + i * NSC_THREADS, kr = idx >> 4, c8 = idx & 15;
+      nsm_load8(X + (int64_t)(kc * 64 + kr) * c + col_base + c8 * 8, true, u[i], v[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+      const int idx = tid + i * NSC_THREADS, kr = idx >> 4, c8 = idx & 15;
+      uint4 hi, lo;
+      nsm_split8(u[i], v[i], hi, lo);
+      const uint32_t off = (c8 >> 3) * (64 * 128) + sw128_offset(kr, c8 & 7);
+      *reinterpret_cast<uint4*>(xs + off) = hi;
+      *reinterpret_cast<uint4*>(xs + L::XCH + off) = lo;
+    }
   };
 
   // ---- X_0: Gram operand from global (rows 0..R-1, the CTA's 128 columns)
@@ -540,7 +561,7 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
     const bool last = it + 1 == iters;
     // ---- 1. B = nc A A^T + nb A
     {
-      constexpr int ITEMS = R * (R / 8), BATCH = (ITEMS / NSC_THREADS) % 9 == 0 ? 9 : 8;
+      constexpr int ITEMS = R * (R / 8), BATCH = (ITEMS / NSC_THREADS) % 6 == 0 ? 6 : 4;
       static_assert(ITEMS % (NSC_THREADS * BATCH) == 0, "staging batches");
       for (int i0 = 0; i0 < ITEMS / NSC_THREADS; i0 += BATCH) {
         float4 u[BATCH], v[BATCH];
@@ -579,6 +600,10 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
       }
       __syncwarp();
     }
+    // the first two X chunks of step 2 do not depend on B: stage them while the MMAs run
+    // (the stages' previous MMAs completed before the last iteration's epilogue)
+    stage_x(0, 0);
+    if (L::KB > 1) stage_x(1, 1);
     wait_bar(mbar, mph);
     // B rows -> K-major operand in place of A's.  The b A term takes A = hi + lo
     // (within 2^-17 relative) from the operand itself: each thread reads exactly
@@ -608,30 +633,16 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     // ---- 2. X_j <- B X_j + a X_j: X rows in 64-row chunks (MN-major [64 k][128 n]) through two stages
+#pragma unroll 1
     for (int kc = 0; kc < L::KB; ++kc) {
       const int st = kc & 1;
       uint8_t* xs = xst + st * L::XSTAGE;
-      if (kc >= 2) wait_bar(xbar + st, st ? xph1 : xph0);  // chunk kc - 2's MMAs released the stage
-      {
-        constexpr int ITEMS = 64 * (NSC_COLS / 8), IT = ITEMS / NSC_THREADS;
-        float4 u[IT], v[IT];
-#pragma unroll
-        for (int i = 0; i < IT; ++i) {
-          const int idx = tid + i * NSC_THREADS, kr = idx >> 4, c8 = idx & 15;
-          nsm_load8(X + (int64_t)(kc * 64 + kr) * c + col_base + c8 * 8, true, u[i], v[i]);
-        }
-#pragma unroll
-        for (int i = 0; i < IT; ++i) {
-          const int idx = tid + i * NSC_THREADS, kr = idx >> 4, c8 = idx & 15;
-          uint4 hi, lo;
-          nsm_split8(u[i], v[i], hi, lo);
-          const uint32_t off = (c8 >> 3) * (64 * 128) + sw128_offset(kr, c8 & 7);
-          *reinterpret_cast<uint4*>(xs + off) = hi;
-          *reinterpret_cast<uint4*>(xs + L::XCH + off) = lo;
-        }
+      if (kc >= 2) {
+        wait_bar(xbar + st, st ? xph1 : xph0);  // chunk kc - 2's MMAs released the stage
+        stage_x(kc, st);
+        fence_async_smem();
+        __syncthreads();
       }
-      fence_async_smem();
-      __syncthreads();
       if (ok && issuer) {
         tc_fence_after();
         if (elect_one()) {
@@ -650,19 +661,20 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
         __syncwarp();
       }
     }
-    // X values of the tile-0 row of this thread (the a X term), loaded while the MMAs finish
-    float xpre[64];
-    {
-      const float4* xr = reinterpret_cast<const float4*>(X + (int64_t)tile_row(0) * c + col_base + half * 64);
+    // The a X term: X is read in 32 x 32 blocks with coalesced 16-byte loads
+    // (lane -> row 4k + lane / 8, columns 4 (lane % 8)) and turned into rows
+    // through the warp's transpose buffer; X' leaves the same way.  Buffer row
+    // stride 36 floats: conflict-free in both directions.  The first block's
+    // loads are issued while the MMAs finish.
+    auto load_blk = [&](int t, int c0, float4 (&xl)[8]) {
+      const int rbase = tile_row(t) - lane;  // first row of this warp's 32
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float4 a4 = xr[e];
-        xpre[4 * e] = a4.x;
-        xpre[4 * e + 1] = a4.y;
-        xpre[4 * e + 2] = a4.z;
-        xpre[4 * e + 3] = a4.w;
-      }
-    }
+      for (int k = 0; k < 8; ++k)
+        xl[k] = *reinterpret_cast<const float4*>(X + (int64_t)(rbase + 4 * k + (lane >> 3)) * c + col_base + c0 +
+                                                 (lane & 7) * 4);
+    };
+    float4 xl[8];
+    load_blk(0, half * 64, xl);
     // the last chunk's commit covers every MMA of the product
     {
       const int st = (L::KB - 1) & 1;
@@ -679,23 +691,28 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
     for (int t = 0; t < L::NMT; ++t) {
       if (!tile_has(t)) continue;
       const int row = tile_row(t);
-      float* xr = X + (int64_t)row * c + col_base;
-      if (t > 0) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float4 a4 = reinterpret_cast<const float4*>(xr + half * 64)[e];
-          xpre[4 * e] = a4.x;
-          xpre[4 * e + 1] = a4.y;
-          xpre[4 * e + 2] = a4.z;
-          xpre[4 * e + 3] = a4.w;
-        }
-      }
+      const int rbase = row - lane;
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const int c0 = half * 64 + h2 * 32;
+        // block -> rows
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<float4*>(tbuf + (4 * k + (lane >> 3)) * 36 + (lane & 7) * 4) = xl[k];
+        __syncwarp();
         float x[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = xpre[h2 * 32 + e];
+        for (int e = 0; e < 32; e += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(tbuf + lane * 36 + e);
+          x[e] = a4.x;
+          x[e + 1] = a4.y;
+          x[e + 2] = a4.z;
+          x[e + 3] = a4.w;
+        }
+        // next block's loads in flight while this one is computed
+        if (h2 == 0) load_blk(t, c0 + 32, xl);
+        else if (t + 1 < L::NMT && tile_has(t + 1)) load_blk(t + 1, half * 64, xl);
         uint32_t v[32];
         if (ok) {
           tmem_ld32(tmem + lane_base + t * NSC_COLS + c0, v);
@@ -706,22 +723,17 @@ __global__ void __launch_bounds__(NSC_THREADS, 1)
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[e] = fmaf(na, x[e], __uint_as_float(v[e]));
-        // X' rows leave through the warp's 32 x 32 transpose buffer (row stride 36
-        // floats: conflict-free both ways), so that each store writes 4 whole
-        // 128-byte row segments instead of 32 scattered 16-byte pieces
+        // rows -> block, whole 128-byte row segments per store
         __syncwarp();
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
           *reinterpret_cast<float4*>(tbuf + lane * 36 + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
         __syncwarp();
-        {
-          const int rbase = row - lane;  // first row of this warp's 32
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int rr = 4 * k + (lane >> 3), cc = (lane & 7) * 4;
-            *reinterpret_cast<float4*>(X + (int64_t)(rbase + rr) * c + col_base + c0 + cc) =
-                *reinterpret_cast<const float4*>(tbuf + rr * 36 + cc);
-          }
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3), cc = (lane & 7) * 4;
+          *reinterpret_cast<float4*>(X + (int64_t)(rbase + rr) * c + col_base + c0 + cc) =
+              *reinterpret_cast<const float4*>(tbuf + rr * 36 + cc);
         }
         if (!last) nsc_put_row32<L::ROWBLK, L::PART>(opa, row, c0, x);
       }
