@@ -260,21 +260,19 @@ __global__ void k_transpose_batch(const float* __restrict__ X, float* __restrict
   }
 }
 
-}  // namespace ttt
-
-namespace ttt {
-
 // ---------------------------------------------------------------------------
 // The whole Newton-Schulz loop of one matrix in one launch (bf16 mode).
 //
-// A cluster of CS = c / 128 CTAs per matrix; CTA j owns columns
+// The quintic's coefficients (a, b, c) are na, nb_, nc here (c is the column
+// count).  A cluster of CS = c / 128 CTAs per matrix; CTA j owns columns
 // [128 j, 128 j + 128) of the wide iterate X (R x c, R in {128, 192}), which is
 // updated in place in global memory.  With A = X X^T kept in global memory
 // (R x R), one iteration is, in every CTA:
-//   1. B = cc A A^T + b A, computed whole by each CTA (K = R, both operands are
-//      A's rows, resident in shared memory; A is symmetric up to rounding);
-//   2. X_j <- B X_j + a X_j for its own columns (K = R in 64-row chunks through
-//      two staging buffers);
+//   1. B = nc A A^T + nb_ A, computed whole by each CTA (K = R, both operands
+//      are A's rows, resident in shared memory; A is symmetric up to rounding);
+//   2. X_j <- B X_j + na X_j for its own columns (K = R in 64-row chunks
+//      through two staging buffers; the first two are staged while step 1's
+//      MMAs run);
 //   3. unless it is the last iteration: P_j = X_j X_j^T (K = 128) into an fp32
 //      shared tile; cluster barrier; CTA j sums the rows i = j (mod CS) of
 //      A = sum_q P_q over q = 0..CS-1 in that fixed order, reading the other
