@@ -486,6 +486,134 @@ __global__ void __launch_bounds__(256, 2) k_shortconv_band(const T* __restrict__
   }
 }
 
+// bf16 variant.  Each thread computes two horizontally adjacent outputs of one
+// 8-channel chunk, so a chunk loaded from shared memory serves up to three taps
+// of both; band rows carry a zero slot on each side (and one past an odd width),
+// so the tap loop has no bounds tests; bf16 -> fp32 by a shift or a mask, and
+// packed fp32x2 FMAs.  The sums are the same as k_shortconv_band's, in the same
+// order (a tap outside the frame adds w * 0).
+constexpr int CONV2_SX = 2;  // outputs per thread along x
+__host__ __device__ constexpr int conv2_row_slots(int gw) { return (gw + CONV2_SX - 1) / CONV2_SX * CONV2_SX + 2; }
+__host__ __device__ constexpr size_t conv2_band_bytes(int BR, int gw) {
+  return (size_t)(BR + 2) * conv2_row_slots(gw) * CONV_GROUP * 2;
+}
+__host__ __device__ constexpr size_t conv2_band_smem(int BR, int gw) {
+  return 9 * CONV_GROUP * sizeof(float) + 2 * conv2_band_bytes(BR, gw);
+}
+
+// 8 bf16 (one 16-byte chunk) -> 4 fp32 pairs
+__device__ __forceinline__ void bf16x8_f2(const uint4 q, float2 (&f)[4]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) f[e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+}
+
+__global__ void __launch_bounds__(256, 2) k_shortconv_band2(const __nv_bfloat16* __restrict__ V, int64_t ldv,
+                                                         __nv_bfloat16* __restrict__ out, int64_t ldo,
+                                                         const float* __restrict__ taps, int N, int gh, int gw, int C,
+                                                         int act, int BR) {
+  constexpr int TPT = CONV_GROUP / 8;  // threads (8-channel chunks) per token
+  constexpr int NL = 256 / TPT;        // output pairs per pass
+  extern __shared__ __align__(16) uint8_t cdyn[];
+  float* wt = reinterpret_cast<float*>(cdyn);  // [9][CONV_GROUP]
+  uint8_t* bufs = cdyn + 9 * CONV_GROUP * sizeof(float);
+  const int RS = conv2_row_slots(gw);
+  const size_t bb = conv2_band_bytes(BR, gw);
+  const int g0 = blockIdx.x * CONV_GROUP;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < 9 * CONV_GROUP; i += 256) {
+    const int k = i / CONV_GROUP, c = i % CONV_GROUP;
+    wt[k * CONV_GROUP + c] = (g0 + c < C) ? taps[(g0 + c) * 9 + k] : 0.f;
+  }
+  const int chunk = tid % TPT, tl = tid / TPT;
+  const int c0 = g0 + chunk * 8;
+  const int ntok = gh * gw, nbands = (gh + BR - 1) / BR, nstrips = (gw + CONV2_SX - 1) / CONV2_SX;
+  __syncthreads();
+  float2 wr[9][4];  // this thread's taps as channel pairs, in registers for all its outputs
+#pragma unroll
+  for (int k = 0; k < 9; ++k)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      wr[k][i] = make_float2(wt[k * CONV_GROUP + chunk * 8 + 2 * i], wt[k * CONV_GROUP + chunk * 8 + 2 * i + 1]);
+  const int rowchunks = RS * TPT;
+  for (int n = blockIdx.y; n < N; n += gridDim.y) {
+    const int64_t frame0 = (int64_t)n * ntok;
+    // band bi: input rows bi*BR - 1 .. bi*BR + BR, slots x = -1 .. RS - 2 (zero outside the frame)
+    auto issue = [&](int bi, uint8_t* buf) {
+      const int y0 = bi * BR - 1;
+      for (int idx = tid; idx < (BR + 2) * rowchunks; idx += 256) {
+        const int r = idx / rowchunks, rem = idx % rowchunks, x = rem / TPT - 1, k = rem % TPT;
+        const int yy = y0 + r, ch = g0 + k * 8;
+        const bool in = yy >= 0 && yy < gh && x >= 0 && x < gw && ch < C;
+        const __nv_bfloat16* src = in ? V + (frame0 + (int64_t)yy * gw + x) * ldv + ch : V;
+        cp_async16_cg(buf + (size_t)idx * 16, src, in ? 16u : 0u);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    __syncthreads();  // taps written; the previous frame's buffers are no longer read
+    issue(0, bufs);
+    for (int bi = 0; bi < nbands; ++bi) {
+      uint8_t* cur = bufs + (bi & 1) * bb;
+      if (bi + 1 < nbands) {
+        issue(bi + 1, bufs + ((bi + 1) & 1) * bb);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      }
+      __syncthreads();
+      const int y0 = bi * BR, rows = min(BR, gh - y0);
+      if (c0 < C) {
+        for (int p = tl; p < rows * nstrips; p += NL) {
+          const int ry = p / nstrips, x0 = (p % nstrips) * CONV2_SX;  // outputs (y0 + ry, x0), (y0 + ry, x0 + 1)
+          float2 a0[4], a1[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a0[i] = a1[i] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int dy = 0; dy < 3; ++dy) {
+            // slots x0 .. x0 + 3 hold inputs x0 - 1 .. x0 + 2 of band row ry + dy
+            const uint4* rp = reinterpret_cast<const uint4*>(cur) + ((size_t)(ry + dy) * RS + x0) * TPT + chunk;
+            float2 in[4];
+            bf16x8_f2(rp[0], in);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a0[i] = __ffma2_rn(wr[dy * 3][i], in[i], a0[i]);
+            bf16x8_f2(rp[TPT], in);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              a0[i] = __ffma2_rn(wr[dy * 3 + 1][i], in[i], a0[i]);
+              a1[i] = __ffma2_rn(wr[dy * 3][i], in[i], a1[i]);
+            }
+            bf16x8_f2(rp[2 * TPT], in);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              a0[i] = __ffma2_rn(wr[dy * 3 + 2][i], in[i], a0[i]);
+              a1[i] = __ffma2_rn(wr[dy * 3 + 1][i], in[i], a1[i]);
+            }
+            bf16x8_f2(rp[3 * TPT], in);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a1[i] = __ffma2_rn(wr[dy * 3 + 2][i], in[i], a1[i]);
+          }
+          if (act == 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              a0[i].x = a0[i].x / (1.0f + expf(-a0[i].x));
+              a0[i].y = a0[i].y / (1.0f + expf(-a0[i].y));
+              a1[i].x = a1[i].x / (1.0f + expf(-a1[i].x));
+              a1[i].y = a1[i].y / (1.0f + expf(-a1[i].y));
+            }
+          }
+          __nv_bfloat16* o = out + (frame0 + (int64_t)(y0 + ry) * gw + x0) * ldo + c0;
+          *reinterpret_cast<uint4*>(o) = make_uint4(pack_bf16x2(a0[0].x, a0[0].y), pack_bf16x2(a0[1].x, a0[1].y),
+                                                    pack_bf16x2(a0[2].x, a0[2].y), pack_bf16x2(a0[3].x, a0[3].y));
+          if (x0 + 1 < gw)
+            *reinterpret_cast<uint4*>(o + ldo) = make_uint4(pack_bf16x2(a1[0].x, a1[0].y), pack_bf16x2(a1[1].x, a1[1].y),
+                                                            pack_bf16x2(a1[2].x, a1[2].y), pack_bf16x2(a1[3].x, a1[3].y));
+        }
+      }
+      __syncthreads();  // `cur` may be refilled by the prefetch of band bi + 2
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Low-precision copies of the fp32 fast weights, laid out for the tensor-core kernels:
 //   Wsh (bf16, apply) and Wsh16 (fp16, gradient) rows [0, Hm): W1 [H][m][d];

@@ -325,6 +325,26 @@ int launch_conv_any(const void* V, int64_t ldv, void* Vout, int64_t ldo, const f
   }
   const dim3 grid((C + CONV_GROUP - 1) / CONV_GROUP, (unsigned)std::min<int64_t>(N, 65535));
   ProfScope ps(TTT_PROF_CONV, s);
+  if (dt == TTT_BF16) {
+    // the two-outputs-per-thread bf16 kernel, same band choice with its padded rows
+    const size_t row2 = (size_t)conv2_row_slots(gw) * CONV_GROUP * 2;
+    int BR2 = 0;
+    for (size_t budget : {(size_t)110 * 1024, (size_t)220 * 1024}) {
+      const int64_t br = (int64_t)((budget - fixed) / (2 * row2)) - 2;
+      if (br >= 1) {
+        BR2 = (int)std::min<int64_t>(br, gh);
+        break;
+      }
+    }
+    if (BR2 >= 1) {
+      const size_t smem = conv2_band_smem(BR2, gw);
+      TTT_CHECK(cudaFuncSetAttribute(k_shortconv_band2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      k_shortconv_band2<<<grid, 256, smem, s>>>((const __nv_bfloat16*)V, ldv, (__nv_bfloat16*)Vout, ldo, taps, (int)N,
+                                                gh, gw, C, act, BR2);
+      TTT_LAUNCHED();
+      return TTT_OK;
+    }
+  }
   if (BR >= 1) {
     const size_t smem = conv_band_smem(BR, gw, esz);
     if (dt == TTT_BF16) {
