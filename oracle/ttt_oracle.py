@@ -26,6 +26,8 @@ other step is written out in the order and notation of the pages:
      Reconstruction with Hybrid Memory, method overview (chunk-wise TTT).
 * gradient additivity over token shards (sum of per-shard gradients)
   -- Scal3R scheme 2 (Global Context Synchronization); VGG-T3 key finding 2.
+* gated output  o_i = RMSNorm(o'_i) * SiLU(W_g o'_i)
+  -- ZipMap key design 3 (the gated unit, second of the three stabilisers).
 
 Readings where the pages are silent or disagree (each is listed again in the
 design notes): minus sign on the dot-product loss; plain sum over tokens (no
@@ -35,7 +37,9 @@ the wide orientation; renorm with the Frobenius norm per matrix per head; a
 step size lr applied after Newton-Schulz (lr = 1 by default); no momentum;
 a second inner step recomputes the gradient at the updated weights; depthwise
 3x3 zero-padded cross-correlation per frame, no bias, optional SiLU; L2 norm
-with max(||x||, 1e-12); chunked order apply-then-update by default.
+with max(||x||, 1e-12); chunked order apply-then-update by default; the
+gate's RMSNorm has no learnable scale and eps = 1e-6, and W_g acts on the
+token's whole output (all heads concatenated), without bias.
 
 Layouts (all numpy float64 here):
   W1, W3: [H, m, d];  W2: [H, d, m]
@@ -300,6 +304,25 @@ def chunked(W: FastWeights, Q, K, V, eta, chunk: int, steps: int, cfg: NSConfig,
             W = update(W, K[c0:c1], V[c0:c1], eta[c0:c1], steps, cfg, qk_l2norm)
             O[c0:c1] = apply(W, Q[c0:c1], qk_l2norm)
     return W, O
+
+
+# ---------------------------------------------------------------------------
+# ZipMap's gated output (key design 3, second stabiliser)
+
+RMS_EPS = 1e-6
+
+
+def rmsnorm(X, eps: float = RMS_EPS) -> np.ndarray:
+    """RMSNorm(x) = x / sqrt(mean(x^2) + eps) over the last axis, no learnable scale."""
+    X = np.asarray(X, dtype=np.float64)
+    return X / np.sqrt(np.mean(X * X, axis=-1, keepdims=True) + eps)
+
+
+def output_gate(Oprime, Wg, eps: float = RMS_EPS) -> np.ndarray:
+    """o_i = RMSNorm(o'_i) * SiLU(W_g o'_i) per token; o' [T, D], W_g [D, D] (no bias)."""
+    Oprime = np.asarray(Oprime, dtype=np.float64)
+    Wg = np.asarray(Wg, dtype=np.float64)
+    return rmsnorm(Oprime, eps) * silu(Oprime @ Wg.T)
 
 
 # ---------------------------------------------------------------------------

@@ -357,3 +357,44 @@ def test_chunked_carry_resumes():
     _, O3 = O.chunked(W, Q, K, V2, eta, chunk=10, steps=1, cfg=cfg)
     np.testing.assert_allclose(O3[:10], Oall[:10], atol=0)
     assert np.abs(O3[10:] - Oall[10:]).max() > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# ZipMap's gated output o = RMSNorm(o') * SiLU(W_g o') (key design 3)
+
+def test_output_gate_hand_worked_identity_gate():
+    # x = [1, -2, 3]: mean(x^2) = 14/3, so RMSNorm(x) = x sqrt(3/14) (eps shifts it by ~1e-7);
+    # logistic values sigma(1), sigma(-2), sigma(3) from tables
+    r = 0.4629100498862757  # sqrt(3/14)
+    s1, sm2, s3 = 0.7310585786300049, 0.11920292202211755, 0.9525741268224334
+    x = np.array([[1.0, -2.0, 3.0]])
+    want = np.array([1.0 * r * (1.0 * s1), -2.0 * r * (-2.0 * sm2), 3.0 * r * (3.0 * s3)])
+    got = O.output_gate(x, np.eye(3))[0]
+    assert np.allclose(got, want, rtol=1e-6, atol=0)
+
+
+def test_output_gate_zero_gate_and_orientation():
+    rng = np.random.default_rng(70)
+    x = rng.standard_normal((5, 6))
+    assert np.array_equal(O.output_gate(x, np.zeros((6, 6))), np.zeros((5, 6)))
+    # W_g maps component 1 to component 0 only: W_g x = [x1, 0, ...] (a transposed
+    # gate would give [0, x0, 0, ...])
+    Wg = np.zeros((6, 6))
+    Wg[0, 1] = 1.0
+    got = O.output_gate(x, Wg)
+    rms = O.rmsnorm(x)
+    assert np.all(got[:, 1:] == 0.0)
+    assert np.allclose(got[:, 0], rms[:, 0] * x[:, 1] / (1.0 + np.exp(-x[:, 1])), rtol=1e-12)
+
+
+def test_output_gate_rmsnorm_is_per_token_and_scale_free():
+    rng = np.random.default_rng(71)
+    x = rng.standard_normal((7, 8))
+    Wg = rng.standard_normal((8, 8))
+    c = np.exp(rng.standard_normal((7, 1)))  # a different positive scale per token
+    # RMSNorm(c x) = RMSNorm(x) per row and W_g/c (c x) = W_g x, up to the eps term
+    a = O.output_gate(x, Wg, eps=0.0)
+    b = np.stack([O.output_gate(c[i] * x[i:i + 1], Wg / c[i], eps=0.0)[0] for i in range(7)])
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+    # each normalised row has mean square 1
+    assert np.allclose(np.mean(O.rmsnorm(x, eps=0.0) ** 2, axis=1), 1.0, rtol=1e-12)
