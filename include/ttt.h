@@ -116,7 +116,11 @@ int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int6
              ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, float* G,
              void* ws, size_t ws_bytes, void* stream);
 
-/* Muon step from a given gradient G (layout as in ttt_grad); updates W in place. */
+/* Muon step from a given gradient G (layout as in ttt_grad); updates W in place.
+ * Newton-Schulz precision: TTT_FP32 multiplies in fp32 on the CUDA cores;
+ * TTT_BF16 multiplies on the tensor cores from split operands (each fp32
+ * value as bf16 hi + bf16 lo, products hi*hi + hi*lo + lo*hi accumulated in
+ * fp32), about 2^-16 relative per product. */
 int ttt_step(ttt_weights W, const float* G, const ttt_ns_cfg* ns, ttt_dims dims, ttt_dtype dtype,
              void* ws, size_t ws_bytes, void* stream);
 
