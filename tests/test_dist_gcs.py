@@ -34,7 +34,7 @@ def _data(H=2, d=6, m=8, T=48, seed=7):
     return W, K, V, Q, eta
 
 
-def _rank_main(rank, world, port, chunk, steps, out_q):
+def _rank_main(rank, world, port, chunk, steps, order, out_q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -64,19 +64,19 @@ def _rank_main(rank, world, port, chunk, steps, out_q):
         def apply(t0, t1):
             outs[t0:t1] = O.apply(state["W"], Ql[t0:t1])
 
-        sharded_layer(per, steps, grad, allreduce, step, apply, chunk=chunk)
+        sharded_layer(per, steps, grad, allreduce, step, apply, chunk=chunk, order=order)
         Wf = state["W"]
         out_q.put((rank, np.concatenate([Wf.W1.ravel(), Wf.W3.ravel(), Wf.W2.ravel()]), outs))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("chunk,steps", [(0, 1), (0, 2), (8, 1)])
-def test_two_rank_gcs_equals_single_process(chunk, steps):
+@pytest.mark.parametrize("chunk,steps,order", [(0, 1, 0), (0, 2, 0), (8, 1, 0), (8, 1, 1)])
+def test_two_rank_gcs_equals_single_process(chunk, steps, order):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, chunk, steps, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, chunk, steps, order, q)) for r in range(2)]
     for p in procs:
         p.start()
     res = {}
@@ -102,8 +102,11 @@ def test_two_rank_gcs_equals_single_process(chunk, steps):
         Or = np.zeros_like(Q)
         for c0 in range(0, per, chunk):
             idx = np.r_[c0:c0 + chunk, per + c0:per + c0 + chunk]
-            Or[idx] = O.apply(Wr, Q[idx])
+            if order == 0:
+                Or[idx] = O.apply(Wr, Q[idx])
             Wr = O.update(Wr, K[idx], V[idx], eta[idx], steps, cfg)
+            if order == 1:
+                Or[idx] = O.apply(Wr, Q[idx])
     wr = np.concatenate([Wr.W1.ravel(), Wr.W3.ravel(), Wr.W2.ravel()])
     np.testing.assert_allclose(res[0][0], wr, rtol=0, atol=1e-10)
     np.testing.assert_allclose(np.vstack([res[0][1], res[1][1]]), Or, rtol=0, atol=1e-10)
