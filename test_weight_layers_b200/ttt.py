@@ -205,11 +205,11 @@ def host_buffer(dm: Dims, T: int, dtype: int, conv: bool = False, device="cuda")
 
 def ttt_layer_host(W: Weights, hQ, hK, hV, hEta, hO, T, chunk, order, steps, ns: NSCfg, dm: Dims, io: IOCfg, dbuf,
                    ws, taps=None, grid_h=0, grid_w=0, stream=None):
-    """hQ, hK, hV, hEta, hO are host (pinned CPU) tensors; dbuf, ws, taps and W are on the device."""
+    """hQ, hK, hV, hEta, hO are host (pinned CPU) tensors; dbuf, ws, taps and W are on the device.
+    chunk > 0 runs the causal carry in the given order (0 apply then update, 1 update then apply)."""
     _check("ttt_layer_host", lib().ttt_layer_host(
         W, _ptr(hQ), _ptr(hK), _ptr(hV), _ptr(hEta), _ptr(hO), T, chunk, order, steps, ctypes.byref(ns), _ptr(taps),
-        grid_h,
-        grid_w, dm, ctypes.byref(io), dtype_code(hQ.dtype), _ptr(dbuf), dbuf.numel(), _ptr(ws), ws.numel(),
+        grid_h, grid_w, dm, ctypes.byref(io), dtype_code(hQ.dtype), _ptr(dbuf), dbuf.numel(), _ptr(ws), ws.numel(),
         _stream(stream)))
 
 
