@@ -398,3 +398,86 @@ def test_output_gate_rmsnorm_is_per_token_and_scale_free():
     assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
     # each normalised row has mean square 1
     assert np.allclose(np.mean(O.rmsnorm(x, eps=0.0) ** 2, axis=1), 1.0, rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# which orthogonalised gradient goes to which matrix (ZipMap key design 3),
+# the second inner step (VGG-T3 key design 3), and which tensor ShortConv2D
+# acts on (VGG-T3 key design 2)
+
+
+def _rank1(rng, r, c):
+    return np.outer(rng.normal(size=r), rng.normal(size=c))
+
+
+def test_muon_step_pairs_each_gradient_with_its_own_matrix(golden):
+    # Rank-1 gradients have the closed form NS(g) = phi(1) g / ||g|| (phi(1) from the
+    # scalar iterates), so each updated matrix follows from its own gradient alone.
+    rng = np.random.default_rng(81)
+    H, d, m = 2, 5, 9
+    W = rand_weights(H, d, m, rng)
+    G = O.FastWeights(np.stack([_rank1(rng, m, d) for _ in range(H)]),
+                      np.stack([_rank1(rng, m, d) for _ in range(H)]),
+                      np.stack([_rank1(rng, d, m) for _ in range(H)]))
+    cfg = O.NSConfig()
+    phi1 = float(golden("ns_scalar.txt")[-1][1])
+    out = O.muon_step(W, G, cfg)
+    for name in ("W1", "W3", "W2"):
+        for h in range(H):
+            w = getattr(W, name)[h]
+            g = getattr(G, name)[h]
+            step = w - phi1 * g / np.linalg.norm(g)
+            want = np.linalg.norm(w) * step / np.linalg.norm(step)
+            np.testing.assert_allclose(getattr(out, name)[h], want, rtol=0, atol=2e-6, err_msg=f"{name}[{h}]")
+    # a gradient in one matrix moves that matrix only: NS(0) = 0 leaves the others as they were
+    for only in ("W1", "W3", "W2"):
+        Z = O.FastWeights(np.zeros_like(W.W1), np.zeros_like(W.W3), np.zeros_like(W.W2))
+        getattr(Z, only)[:] = getattr(G, only)
+        res = O.muon_step(W, Z, cfg)
+        for name in ("W1", "W3", "W2"):
+            same = np.allclose(getattr(res, name), getattr(W, name), rtol=0, atol=1e-14)
+            assert same == (name != only), (only, name)
+
+
+def test_two_inner_steps_recompute_the_gradient_at_the_updated_weights():
+    # steps = 2 is one step, then another from the weights the first produced; reusing the
+    # first gradient for the second step gives a different result.
+    W, K, V, eta = _update_inputs(H=2, d=6, m=8, T=24, rng=np.random.default_rng(82))
+    cfg = O.NSConfig()
+    two = O.update(W, K, V, eta, 2, cfg)
+    once = O.update(W, K, V, eta, 1, cfg)
+    twice = O.update(once, K, V, eta, 1, cfg)
+    for name in ("W1", "W3", "W2"):
+        np.testing.assert_allclose(getattr(two, name), getattr(twice, name), rtol=0, atol=1e-13)
+    Kh = O.l2norm_heads(K, 2, 6)
+    g0 = O.grad(W, Kh, V, eta)
+    stale = O.muon_step(O.muon_step(W, g0, cfg), g0, cfg)
+    assert np.abs(stale.W1 - two.W1).max() > 1e-3
+    # the second step's gradient is the gradient at the once-updated weights
+    g1 = O.grad(once, Kh, V, eta)
+    assert np.abs(g1.W2 - g0.W2).max() > 1e-3 * np.abs(g0.W2).max()
+
+
+def test_shortconv_acts_on_values_only():
+    # VGG-T3 key design 2: the regression target becomes K -> V' = ShortConv2D(V); K is only
+    # L2-normalised.  So the update with the conv equals the update on a pre-convolved V.
+    rng = np.random.default_rng(83)
+    H, d, m, N, gh, gw = 2, 4, 8, 2, 3, 4
+    T = N * gh * gw
+    W = rand_weights(H, d, m, rng)
+    K = rng.normal(size=(T, H * d))
+    V = rng.normal(size=(T, H * d))
+    eta = rng.uniform(0.05, 1.0, size=(T, H))
+    taps = rng.normal(size=(H * d, 3, 3)) / 3.0
+    cfg = O.NSConfig()
+    for act in (0, 1):
+        with_conv = O.update(W, K, V, eta, 1, cfg, conv=(taps, N, gh, gw, act))
+        Vp = O.shortconv2d(V, taps, N, gh, gw, act)
+        pre = O.update(W, K, Vp, eta, 1, cfg)
+        for name in ("W1", "W3", "W2"):
+            np.testing.assert_allclose(getattr(with_conv, name), getattr(pre, name), rtol=0, atol=1e-13)
+        # and the conv does change the result (it is not a no-op on these inputs)
+        plain = O.update(W, K, V, eta, 1, cfg)
+        assert np.abs(plain.W2 - with_conv.W2).max() > 1e-3
+    Kh, Vh = O.prepare_kv(K, V, H, d, True, (taps, N, gh, gw, 0))
+    np.testing.assert_allclose(Kh, O.l2norm_heads(K, H, d), rtol=0, atol=0)
