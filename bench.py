@@ -38,6 +38,8 @@ METRIC = "TTT-layer tokens/sec (update+apply) and % of B200 bf16 tensor peak"
 UNIT = "tokens/s"
 L2_BYTES = 126 << 20
 L2_FLUSH_BYTES = 512 << 20
+UPDATE_OPERANDS = ("fp16 tensor-core operands: K^ (normalised), V' = -2^8 eta v (one rounding), fast-weight copy, "
+                   "dH and u (fp32 accumulation)")
 
 
 def parse():
@@ -398,6 +400,18 @@ def run_ours(args, cfg):
     flops_layer = cfg.update_flops() + cfg.apply_flops()
     tflops = flops_layer * world / (ms / 1e3) / 1e12
 
+    # The denominator follows the clocks this run earned: a short timed region at
+    # (near) maximum SM clock is a burst, so it is compared with the burst GEMM
+    # peak; a long or power-capped one with the sustained peak.  Both fractions
+    # are printed.
+    region_s = ms * args.steps / 1e3
+    at_max = bool(clk and clk.get("sm_mhz") and clk.get("sm_max_mhz")
+                  and clk["sm_mhz"] >= 0.95 * clk["sm_max_mhz"])
+    use_burst = region_s < 1.0 and at_max
+    peak_tf = peaks["bf16_tflops"] if use_burst else peaks["bf16_tflops_sustained"]
+    peak_kind = (f"{'burst' if use_burst else 'sustained'} ({peaks['source']}): timed region {region_s:.2f} s, "
+                 f"median SM clock {clk.get('sm_mhz') if clk else None} of {clk.get('sm_max_mhz') if clk else None} MHz")
+
     # dominant kernel: the tensor-core gradient kernel
     g_ms, g_n = prof["grad"]
     tok_per_launch = Tn if not cfg.chunk else cfg.chunk
@@ -405,10 +419,10 @@ def run_ours(args, cfg):
     roof = None
     if g_n and dcode == T.TTT_BF16:
         ach = grad_flops / (g_ms / g_n / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
+                "frac_of_burst": ach / peaks["bf16_tflops"], "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
                 "traffic": traffic_per_launch(tok_per_launch), "kernel": "k_update_grad_tc",
-                "peak_kind": f"fp16/bf16 dense (same tensor rate), sustained, {peaks['source']}",
+                "peak_kind": "fp16/bf16 dense (same tensor rate), " + peak_kind,
                 "launch_ms": g_ms / g_n}
     elif g_n:
         # fp32 mode: CUDA-core FMA pipe, 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz
@@ -426,8 +440,12 @@ def run_ours(args, cfg):
                                       if flush is None else
                                       f"inputs fit in L2: {L2_FLUSH_BYTES >> 20} MB written before every step, "
                                       "outside its events"),
-            "tflops": tflops, "frac_of_bf16_peak": tflops * 1e12 / world / (peaks["bf16_tflops_sustained"] * 1e12),
-            "update_operands": "fp16 (exact from bf16 inputs)" if dcode == T.TTT_BF16 else "fp32",
+            "tflops": tflops,
+            "layer_frac_of_bf16_peak": {"frac": tflops / world / peak_tf,
+                                        "frac_of_burst": tflops / world / peaks["bf16_tflops"],
+                                        "frac_of_sustained": tflops / world / peaks["bf16_tflops_sustained"],
+                                        "peak_kind": peak_kind},
+            "update_operands": UPDATE_OPERANDS if dcode == T.TTT_BF16 else "fp32",
             "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clk}
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region

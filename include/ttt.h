@@ -158,6 +158,10 @@ int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
  *    order them on one stream.
  *  - A device-side wait that times out cannot be polled here (there is no
  *    workspace); O is then undefined.
+ *  - The looked-up address is kept for the life of the process: after
+ *    cudaDeviceReset on a device, this entry point (like ttt_layer_host, whose
+ *    copy streams and events are kept per device) must not be called again on
+ *    that device.
  * Arguments and layouts as for ttt_apply, minus the workspace. */
 #define TTT_NOALLOC_SCRATCH_BYTES (8u << 20)
 int ttt_apply_noalloc(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
@@ -212,6 +216,15 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
  * following ttt_poll_status reports TTT_ERR_TIMEOUT until ttt_reset_status.
  * timeout_us must be in [1, 10^7]. */
 int ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned timeout_us, void* stream);
+
+/* Target the library's kernels were compiled for, from the compiler's
+ * architecture list (1000 for sm_100a); needs no GPU. */
+int ttt_compiled_arch(void);
+
+/* Binary version the CUDA runtime reports for the library's kernels on the
+ * current device (major * 10 + minor: 100 for sm_100a) into *version.
+ * Returns TTT_ERR_CUDA without a usable device. */
+int ttt_kernel_binary_version(int* version);
 
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(int status);

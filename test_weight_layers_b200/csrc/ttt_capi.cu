@@ -1190,6 +1190,22 @@ int ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned timeout_us, vo
   return TTT_OK;
 }
 
+int ttt_compiled_arch(void) {
+#ifdef __CUDA_ARCH_LIST__
+  return __CUDA_ARCH_LIST__;
+#else
+  return 0;
+#endif
+}
+
+int ttt_kernel_binary_version(int* version) {
+  if (!version) return TTT_ERR_INVALID;
+  cudaFuncAttributes a{};
+  TTT_CHECK(cudaFuncGetAttributes(&a, k_selftest_wait));
+  *version = a.binaryVersion;
+  return TTT_OK;
+}
+
 const char* ttt_status_string(int status) {
   switch (status) {
     case TTT_OK: return "ok";

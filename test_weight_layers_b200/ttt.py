@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "ttt_layer_host": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), P, I, I, Dims,
                                    ctypes.POINTER(IOCfg), I, P, SZ, P, SZ, P]),
             "ttt_status_string": (ctypes.c_char_p, [I]),
+            "ttt_compiled_arch": (I, []),
+            "ttt_kernel_binary_version": (I, [ctypes.POINTER(I)]),
             "ttt_selftest_wait_timeout": (I, [P, SZ, ctypes.c_uint, P]),
             "ttt_launch_count": (ctypes.c_uint64, []),
             "ttt_profile_enable": (I, [I]),

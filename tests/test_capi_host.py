@@ -37,9 +37,8 @@ def test_library_exports_every_declared_symbol(lib):
         assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
 
 
-def test_library_is_built_for_sm100a():
-    out = os.popen(f"strings -a {B.LIB} | grep -c sm_100a").read().strip()
-    assert int(out or 0) > 0
+def test_library_is_built_for_sm100a(lib):
+    assert lib.ttt_compiled_arch() == 1000
 
 
 def test_status_strings(lib):

@@ -1,5 +1,6 @@
 """GPU parity of each entry point against the fp64 oracle at small sizes
 (several 128-token tiles plus a ragged tail), through the C ABI."""
+import ctypes
 import numpy as np
 import pytest
 import torch
@@ -201,3 +202,9 @@ def test_device_wait_timeout_is_reported_and_context_survives():
     T.ttt_apply(W.abi, Q, O_, 256, dm, T.io_cfg(), ws)
     check_status(ws)
     assert rel_fro(f64(O_), O.apply(W.oracle(), f64(Q))) < 1e-2
+
+
+def test_kernels_run_as_sm100a_binaries():
+    v = ctypes.c_int(0)
+    assert T.lib().ttt_kernel_binary_version(ctypes.byref(v)) == T.TTT_OK
+    assert v.value == 100
