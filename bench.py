@@ -169,7 +169,9 @@ def oracle_sample_times(cfg, sample):
     t1 = time.perf_counter()
     Wn = O.muon_step(W, G, ns)
     t2 = time.perf_counter()
-    O.apply(Wn, Q)
+    Oq = O.apply(Wn, Q)
+    if cfg.gate:
+        O.output_gate(Oq, inp.gate_weight().double().numpy())
     t3 = time.perf_counter()
     return (t1 - t0) / sample, (t3 - t2) / sample, (t2 - t1)
 
@@ -233,7 +235,8 @@ def workload_config(cfg, n, l2_note):
                          f"step(s){', ShortConv2D on V' if cfg.conv else ''}"
                          f"{f', {cfg.n_chunks} causal chunks of {cfg.chunk} (' if cfg.chunk else ''}"
                          f"{('update then apply)' if cfg.order else 'apply then update)') if cfg.chunk else ''}, "
-                         f"apply on {cfg.apply_tokens} tokens"),
+                         f"apply on {cfg.apply_tokens} tokens"
+                         f"{', gated output RMSNorm(o) SiLU(W_g o)' if cfg.gate else ''}"),
             "tokens_per_gpu": cfg.tokens, "heads": cfg.heads, "d": cfg.d, "m": cfg.m, "inner_steps": cfg.steps,
             "chunk": cfg.chunk or None, "order": cfg.order if cfg.chunk else None, "qk_l2norm": True,
             "l2": l2_note,
@@ -316,6 +319,10 @@ def run_ours(args, cfg):
     taps = S.conv_taps(cfg.seed, D).to(dev) if cfg.conv else None
     Vc = torch.empty_like(V) if cfg.conv else None
     O = torch.empty((Ta, D), dtype=tdt, device=dev)
+    # gated output (ZipMap): the apply writes O' and the gate writes the layer output
+    Wg = S.gate_weight(cfg.seed, D).to(dev) if cfg.gate else None
+    Og = torch.empty_like(O) if cfg.gate else None
+    gws = T.gate_workspace(Ta, D, device=dev) if cfg.gate else None
     G = torch.empty(3 * H * m * d, dtype=torch.float32, device=dev)
     ws = T.workspace(dm, cfg.chunk or max(Tn, Ta), dcode, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -330,6 +337,8 @@ def run_ours(args, cfg):
         if world == 1 and not cfg.chunk:
             T.ttt_update(Wabi, Kx, Vuse, ex, Tn, cfg.steps, ns, dm, io, ws)
             T.ttt_apply(Wabi, Qx, Ox, Ta, dm, io, ws)
+            if cfg.gate:
+                T.ttt_output_gate(Ox, Wg, Og, Ta, D, gws)
         elif world == 1:
             T.ttt_chunked(Wabi, Qx, Kx, Vuse, ex, Ox, Tn, cfg.chunk, cfg.order, cfg.steps, ns, dm, io, ws)
         else:
@@ -343,6 +352,8 @@ def run_ours(args, cfg):
                 chunk=cfg.chunk, order=cfg.order)
             if not cfg.chunk:
                 T.ttt_apply(Wabi, Qx, Ox, Ta, dm, io, ws)
+                if cfg.gate:
+                    T.ttt_output_gate(Ox, Wg, Og, Ta, D, gws)
 
     def barrier():
         if world > 1:
@@ -419,9 +430,11 @@ def run_ours(args, cfg):
     roof = None
     if g_n and dcode == T.TTT_BF16:
         ach = grad_flops / (g_ms / g_n / 1e3) / 1e12
+        wide = d % 256 == 0 and m % 256 == 0 and d >= 256
         roof = {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
                 "frac_of_burst": ach / peaks["bf16_tflops"], "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
-                "traffic": traffic_per_launch(tok_per_launch), "kernel": "k_update_grad_tc",
+                "traffic": None if wide else traffic_per_launch(tok_per_launch),
+                "kernel": ("k_wgemm gradient products with k_prep_wide (2-SM pairs)" if wide else "k_update_grad_tc"),
                 "peak_kind": "fp16/bf16 dense (same tensor rate), " + peak_kind,
                 "launch_ms": g_ms / g_n}
     elif g_n:
@@ -458,7 +471,7 @@ def run_ours(args, cfg):
         bytes_in = sum(x.numel() * x.element_size() for x in (hK, hV, hQ, he))
         bytes_out = hO.numel() * hO.element_size()
 
-        if world == 1 and Ta == Tn:
+        if world == 1 and Ta == Tn and not cfg.gate:
             # the library's host-buffer entry point: copies overlapped with the computation
             dbuf = T.host_buffer(dm, Tn, dcode, conv=cfg.conv, device=dev)
 
@@ -476,7 +489,7 @@ def run_ours(args, cfg):
                 Q.copy_(hQ, non_blocking=True)
                 eta.copy_(he, non_blocking=True)
                 layer(K, V, Q, eta, O)
-                hO.copy_(O, non_blocking=True)
+                hO.copy_(Og if cfg.gate else O, non_blocking=True)
             e2e_api = "device entry points with torch copies before and after"
 
         e2e_step()

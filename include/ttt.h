@@ -38,8 +38,29 @@
  *    In TTT_BF16 mode the GEMMs read a bfloat16 copy of W that the library
  *    writes into the workspace at the start of each call; W itself stays fp32.
  *  - TTT_BF16 mode runs the tensor-core path and needs d in {128, 192} and
- *    m a multiple of 64; TTT_FP32 mode runs fp32 CUDA-core kernels for any
- *    d <= 256 and m a multiple of 32.  Other shapes return TTT_ERR_UNSUPPORTED.
+ *    m a multiple of 64 (fused kernels), or d and m multiples of 256 (the
+ *    wide-head path for heads such as ZipMap's single head of d = 1024,
+ *    m = 2048: the same arithmetic as separate 2-SM tensor-core products with
+ *    fp16 intermediates in the workspace); TTT_FP32 mode runs fp32 CUDA-core
+ *    kernels for any d <= 256 and m a multiple of 32.  Other shapes return
+ *    TTT_ERR_UNSUPPORTED.
+ *  - Operand range of the TTT_BF16 update (ttt_grad, ttt_update, ttt_chunked,
+ *    ttt_layer_host).  The gradient GEMMs run on fp16 operands with fp32
+ *    accumulation: k^ (k / ||k|| with qk_l2norm = 1, else k itself),
+ *    V' = -s eta v with a power of two s chosen per call so that
+ *    s * max|eta| lies in [16, 32) (for ttt_layer_host with chunk = 0: one s
+ *    for all T tokens), the fp16 copy of W, and dL/dh, u scaled by s.  So
+ *    the scale of eta does not matter; what must hold is that each of these
+ *    stays below fp16's 65504: without the key norm every key element |k|;
+ *    every |V'_t| = s |eta_t| |v_t| < 32 |v_t| |eta_t| / max|eta| (so
+ *    |v| < 2047 always suffices); and u = SiLU(W1 k^) o (W3 k^) and s dL/dh,
+ *    which for normalised keys and weights of the initial scale stay far
+ *    below it (without the key norm, u grows like |k|^2).  Without the key
+ *    norm, key elements below 2^-14 in magnitude lose precision (fp16
+ *    subnormals).  Beyond the range the gradient comes out non-finite: the
+ *    call still returns TTT_OK (it is asynchronous), ttt_poll_status then
+ *    reports TTT_ERR_RANGE, and the Muon step leaves W unchanged (ttt_grad
+ *    returns the non-finite G as is).
  *  - No entry point falls back to the CPU.
  */
 #ifndef TTT_H
@@ -60,7 +81,9 @@ typedef enum {
   TTT_ERR_CUDA = -4,         /* a CUDA runtime call or kernel launch failed */
   TTT_ERR_TIMEOUT = -5,      /* a device-side wait gave up (reported through ttt_poll_status) */
   TTT_ERR_ALIGN = -6,        /* pointer or row stride violates the 16-byte alignment rule */
-  TTT_ERR_SCRATCH = -7       /* problem too large for the fixed scratch of ttt_apply_noalloc */
+  TTT_ERR_SCRATCH = -7,      /* problem too large for the fixed scratch of ttt_apply_noalloc */
+  TTT_ERR_RANGE = -8         /* the gradient came out non-finite: an fp16 operand of the tensor-core
+                                update was out of range (reported through ttt_poll_status) */
 } ttt_status;
 
 typedef enum { TTT_FP32 = 0, TTT_BF16 = 1 } ttt_dtype;
@@ -92,7 +115,9 @@ size_t ttt_workspace_bytes(ttt_dims dims, int64_t T, ttt_dtype dtype);
 int ttt_reset_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream` and return the workspace status word: TTT_OK or the
- * first device-side error recorded since the last reset (TTT_ERR_TIMEOUT). */
+ * first device-side error recorded since the last reset (TTT_ERR_TIMEOUT, or
+ * TTT_ERR_RANGE for a non-finite gradient).  While an error is recorded, the
+ * Muon step of every call on this workspace leaves W unchanged. */
 int ttt_poll_status(const void* ws, void* stream);
 
 /* In-place L2 normalisation of X [T][ld]: every (token, head) row of d values
@@ -158,6 +183,8 @@ int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
  *    order them on one stream.
  *  - A device-side wait that times out cannot be polled here (there is no
  *    workspace); O is then undefined.
+ *  - The wide-head shapes (d and m multiples of 256) return TTT_ERR_UNSUPPORTED:
+ *    their apply keeps a per-token intermediate in the workspace.
  *  - The looked-up address is kept for the life of the process: after
  *    cudaDeviceReset on a device, this entry point (like ttt_layer_host, whose
  *    copy streams and events are kept per device) must not be called again on
@@ -166,6 +193,21 @@ int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
 #define TTT_NOALLOC_SCRATCH_BYTES (8u << 20)
 int ttt_apply_noalloc(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,
                       const ttt_io_cfg* io, ttt_dtype dtype, void* stream);
+
+/* Gated output (ZipMap key design 3, the gated unit after the TTT read-out):
+ *     o_t = RMSNorm(o'_t) * SiLU(W_g o'_t),  RMSNorm(x) = x / sqrt(mean(x^2) + 1e-6)
+ * per token over the whole row of D values (all heads), without a learnable
+ * scale and without a bias.
+ *  - Oprime: [T][ld_in] bf16 (D columns used), e.g. the output of ttt_apply;
+ *    O: [T][ld_out] bf16, may not alias Oprime.  ld 0 means D.
+ *  - Wg: float [D][D] row-major, device (row j gives gate j: (W_g o')_j = Wg[j] . o').
+ *  - ws: ttt_gate_workspace_bytes(T, D) bytes, 256-byte aligned: a bf16 copy of
+ *    W_g and the per-token RMS factors.
+ *  - TTT_BF16 only, D a multiple of 256 (the product runs on 2-SM tensor-core
+ *    pairs in 256 x 256 tiles); other cases return TTT_ERR_UNSUPPORTED. */
+size_t ttt_gate_workspace_bytes(int64_t T, int D);
+int ttt_output_gate(const void* Oprime, int64_t ld_in, const float* Wg, void* O, int64_t ld_out, int64_t T, int D,
+                    ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
 /* Causal chunk carry over T tokens in chunks of `chunk` (the last may be shorter).
  * order 0: O_c = f_{W_(c-1)}(Q_c), then W_c = TTTUpdate(W_(c-1); chunk c);
@@ -243,7 +285,7 @@ typedef enum {
   TTT_PROF_GRAD = 0,    /* gradient kernel (tensor-core in bf16 mode) */
   TTT_PROF_APPLY = 1,   /* apply kernel */
   TTT_PROF_NS = 2,      /* Newton-Schulz iterations and the weight step */
-  TTT_PROF_NORM = 3,    /* Q/K row norms and ttt_l2norm */
+  TTT_PROF_NORM = 3,    /* row norms (fp32 mode, ttt_l2norm) and the max |eta| of the bf16 update */
   TTT_PROF_CONV = 4,    /* ShortConv2D */
   TTT_PROF_REDUCE = 5,  /* split-K reduction of the gradient partials */
   TTT_PROF_SHADOW = 6,  /* bf16 copies of the fast weights */

@@ -13,12 +13,46 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
 #include <type_traits>
 
 namespace ttt {
 
-// device status codes (positive; the host maps any nonzero value to TTT_ERR_TIMEOUT)
-enum : unsigned int { DEV_OK = 0, DEV_TIMEOUT = 5 };
+// device status codes (positive; the host maps them to TTT_ERR_TIMEOUT and TTT_ERR_RANGE)
+enum : unsigned int { DEV_OK = 0, DEV_TIMEOUT = 5, DEV_RANGE = 6 };
+
+constexpr int ETA_PARTS = 128;    // partial maxima of |eta| (k_eta_absmax) that fix the value scale
+
+// Power-of-two scale s of the fp16 value operand V' = -s eta v: s * max|eta|
+// lies in [16, 32), so |V'| <= 32 |v| whatever the scale of eta (fp16 holds
+// values up to 65504; its subnormals start at 2^-14), and the scaled dL/du and
+// dL/dh stay clear of fp16 subnormals.  inv_s = 1/s exactly.  A non-finite
+// maximum gives s = 1 (the gradient then comes out non-finite and is reported
+// as out of range).
+__host__ __device__ __forceinline__ void value_scale(float emax, float& s, float& inv_s) {
+  uint32_t bits;
+  memcpy(&bits, &emax, 4);
+  const int eb = (int)((bits >> 23) & 0xffu);  // biased exponent of max|eta|
+  if (eb == 0xff) {
+    s = inv_s = 1.f;
+    return;
+  }
+  // emax in [2^(eb-127), 2^(eb-126))  ->  s = 2^(131 - eb)
+  int e = 131 - (eb > 1 ? eb : 1);
+  e = e < -120 ? -120 : (e > 120 ? 120 : e);
+  const uint32_t sb = (uint32_t)(e + 127) << 23, ib = (uint32_t)(127 - e) << 23;
+  memcpy(&s, &sb, 4);
+  memcpy(&inv_s, &ib, 4);
+}
+
+// max of the ETA_PARTS partial maxima (one warp; every lane gets the result)
+__device__ __forceinline__ float eta_parts_max(const float* __restrict__ part) {
+  float v = 0.f;
+  for (int i = threadIdx.x & 31; i < ETA_PARTS; i += 32) v = fmaxf(v, part[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 
 struct Guard {
   unsigned int* status;        // workspace status word (device)

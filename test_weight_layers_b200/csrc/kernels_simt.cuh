@@ -187,13 +187,14 @@ __global__ void __launch_bounds__(256, 4) k_rownorm(T* X, int64_t ld, int64_t ro
 // ---------------------------------------------------------------------------
 // Update-operand preparation: one pass over K and V that writes the fp16
 // operands of the tensor-core gradient kernel, K^ = k / max(||k||, 1e-12) per
-// head (or k itself) and V' = vscale * eta_(t,h) * v, densely [T][H*d].  The loss is
-// linear in v, so folding the per-token weight (and the gradient's fp16 scale)
-// into V is exact algebra: the forward then yields dL/du = -eta z directly and
-// the gradient of W2 needs no per-token scaling.  bf16 -> fp16 is exact for values
-// in fp16's normal range; fp16 carries three more significand bits than bf16,
-// which the chained Muon updates need.  One warp per token, the whole row loaded
-// before any reduction.
+// head (or k itself) and V' = -s eta_(t,h) v, densely [T][H*d], with the
+// power-of-two value scale s of the call (value_scale: s max|eta| in [16, 32)).
+// The loss is linear in v, so folding the per-token weight and s into V is
+// exact algebra: the forward then yields s dL/du directly and the gradient of
+// W2 needs no per-token scaling.  bf16 -> fp16 is exact for values in fp16's
+// normal range; fp16 carries three more significand bits than bf16, which the
+// chained Muon updates need.  One warp per token, the whole row loaded before
+// any reduction.
 
 __device__ __forceinline__ void store16_h(__half* p, const float (&v)[8]) {
   uint4 x;
@@ -206,10 +207,14 @@ __device__ __forceinline__ void store16_h(__half* p, const float (&v)[8]) {
 
 __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restrict__ K, int64_t ldk,
                                                     const __nv_bfloat16* __restrict__ V, int64_t ldv,
-                                                    const float* __restrict__ eta, float vscale,
+                                                    const float* __restrict__ eta,
+                                                    const float* __restrict__ eta_part,
                                                     __half* __restrict__ Kh, __half* __restrict__ Vh, int64_t rows,
                                                     int H, int d, int l2norm) {
   constexpr int VN = 8;
+  float vscale, inv_unused;  // V' = -s eta v with the value scale s of this call
+  value_scale(eta_parts_max(eta_part), vscale, inv_unused);
+  vscale = -vscale;
   const int lane = threadIdx.x & 31;
   const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -677,8 +682,13 @@ __global__ void __launch_bounds__(256) k_shadow(const float* __restrict__ W1, co
 // Deterministic split-K reduction: G[i] = sum_{s=0..S-1} P[s][i] in that order.
 
 // G = sum over the S split partials (accumulate = 1: G += that sum), fixed order.
-__global__ void k_reduce_splits(const float* __restrict__ P, int S, int64_t n, float* __restrict__ G, int accumulate) {
+// A non-finite entry of G (an fp16 operand of the tensor-core gradient out of
+// range, or non-finite inputs) records DEV_RANGE in the status word; the weight
+// step then leaves W unchanged.
+__global__ void k_reduce_splits(const float* __restrict__ P, int S, int64_t n, float* __restrict__ G, int accumulate,
+                                unsigned int* status) {
   const int64_t n4 = n / 4;
+  bool finite = true;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
     float4 acc = reinterpret_cast<const float4*>(P)[i];
     for (int s = 1; s < S; ++s) {
@@ -689,7 +699,41 @@ __global__ void k_reduce_splits(const float* __restrict__ P, int S, int64_t n, f
       const float4 g = reinterpret_cast<const float4*>(G)[i];
       acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
     }
+    // |x| <= FLT_MAX is false for inf and NaN
+    finite &= fabsf(acc.x) <= 3.402823466e38f && fabsf(acc.y) <= 3.402823466e38f &&
+              fabsf(acc.z) <= 3.402823466e38f && fabsf(acc.w) <= 3.402823466e38f;
     reinterpret_cast<float4*>(G)[i] = acc;
+  }
+  if (!__all_sync(0xffffffffu, finite) && (threadIdx.x & 31) == 0) atomicCAS(status, DEV_OK, (unsigned int)DEV_RANGE);
+}
+
+// Block maxima of |eta| over n values (grid of ETA_PARTS blocks or fewer; the
+// missing parts are written as 0), for the value scale of the gradient kernel.
+__global__ void __launch_bounds__(512) k_eta_absmax(const float* __restrict__ eta, int64_t n, float* __restrict__ part,
+                                                    int nparts) {
+  __shared__ float red[16];
+  float m = 0.f;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n; i += 4 * stride) {
+    const float a = __ldg(eta + i), b = __ldg(eta + i + stride), c = __ldg(eta + i + 2 * stride),
+                d = __ldg(eta + i + 3 * stride);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d))));
+  }
+  for (; i < n; i += stride) m = fmaxf(m, fabsf(__ldg(eta + i)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) {
+      part[blockIdx.x] = m;
+      if (blockIdx.x == 0)
+        for (int p = gridDim.x; p < nparts; ++p) part[p] = 0.f;
+    }
   }
 }
 
@@ -983,10 +1027,14 @@ __global__ void __launch_bounds__(256) k_step_partials(float* W1, float* W3, flo
   }
 }
 
+// W <- sc (W - lr D).  Skipped when the status word holds an error (a gradient
+// out of range or a timed-out wait), so W is never overwritten with garbage.
 __global__ void k_step_apply(float* W1, float* W3, float* W2, const float* __restrict__ Dw, const float* __restrict__ Dt,
-                             int H, int d, int m, float lr, int renorm, const float* __restrict__ parts) {
+                             int H, int d, int m, float lr, int renorm, const float* __restrict__ parts,
+                             const unsigned int* status) {
   pdl_trigger();
   pdl_wait();
+  if (*(volatile const unsigned int*)status != DEV_OK) return;
   const int b = blockIdx.y;
   const int64_t n = (int64_t)m * d, n4 = n / 4;
   float4* w = reinterpret_cast<float4*>(mat_ptr(W1, W3, W2, b, H, n));

@@ -61,8 +61,6 @@ struct UpdLayout {
 };
 
 constexpr int UPD_THREADS = 352;  // warp 0: forward TMA, 1: MMA, 2..9: epilogue, 10: backward TMA
-constexpr float GRAD_SCALE = 256.f;
-constexpr float GRAD_UNSCALE = 1.f / 256.f;
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
@@ -84,9 +82,9 @@ template <int D>
 __global__ void __launch_bounds__(UPD_THREADS, 1)
     k_update_grad_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb,
-                     const __grid_constant__ CUtensorMap tmW, float* __restrict__ partial, int64_t T, int H,
-                     int m,
-                     int tiles_total, int S, unsigned int* status, unsigned long long timeout_ns) {
+                     const __grid_constant__ CUtensorMap tmW, const float* __restrict__ eta_part,
+                     float* __restrict__ partial, int64_t T, int H, int m, int tiles_total, int S,
+                     unsigned int* status, unsigned long long timeout_ns) {
   using L = UpdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -295,6 +293,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
     // ---------------- epilogue warps 2..9
     const int q = warp & 3;            // TMEM lane quarter accessible to this warp
     const int ch = (warp - 2) >> 2;    // which 32-column half of the slice
+    float vscale_unused, inv_vscale;   // the readout undoes the value scale s of V'
+    value_scale(eta_parts_max(eta_part), vscale_unused, inv_vscale);
     const int row = q * 32 + lane;     // token row within the tile / TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     bool ok = true;
@@ -311,10 +311,10 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_n(ffree, 32);  // F may now be overwritten by the next tile's forward
-      // V arrives as -2^8 eta v (the preparation kernel folds the per-token
-      // weight into it), so Z = dL/du scaled by 2^8 (clear of fp16 subnormals) and
-      // dH is scaled the same way; U~ = u, and g2 = V'^T U~ carries the 2^8.  The
-      // gradient readout multiplies by 2^-8, which is exact.
+      // V arrives as V' = -s eta v (the preparation kernel folds the per-token
+      // weight into it), so Z = s dL/du (clear of fp16 subnormals) and dH is
+      // scaled the same way; U~ = u, and g2 = V'^T U~ carries the s.  The
+      // gradient readout multiplies by 1/s, which is exact.
       const float2 half2 = make_float2(0.5f, 0.5f);
       const float2 mhalf2 = make_float2(-0.5f, -0.5f);
       uint32_t p1[16], p3[16], pu[16];
@@ -382,8 +382,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(dst + c0 + j) =
-                make_float4(__uint_as_float(v[j]) * GRAD_UNSCALE, __uint_as_float(v[j + 1]) * GRAD_UNSCALE,
-                            __uint_as_float(v[j + 2]) * GRAD_UNSCALE, __uint_as_float(v[j + 3]) * GRAD_UNSCALE);
+                make_float4(__uint_as_float(v[j]) * inv_vscale, __uint_as_float(v[j + 1]) * inv_vscale,
+                            __uint_as_float(v[j + 2]) * inv_vscale, __uint_as_float(v[j + 3]) * inv_vscale);
         }
       }
       // g2 columns of this slice: block rb holds d rows 64*rb .. 64*rb+127
@@ -399,8 +399,8 @@ __global__ void __launch_bounds__(UPD_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(dst + j) =
-                make_float4(__uint_as_float(v[j]) * GRAD_UNSCALE, __uint_as_float(v[j + 1]) * GRAD_UNSCALE,
-                            __uint_as_float(v[j + 2]) * GRAD_UNSCALE, __uint_as_float(v[j + 3]) * GRAD_UNSCALE);
+                make_float4(__uint_as_float(v[j]) * inv_vscale, __uint_as_float(v[j + 1]) * inv_vscale,
+                            __uint_as_float(v[j + 2]) * inv_vscale, __uint_as_float(v[j + 3]) * inv_vscale);
         }
       }
     }

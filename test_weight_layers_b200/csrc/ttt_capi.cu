@@ -17,6 +17,7 @@
 #include "kernels_nsmma.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
+#include "kernels_wide.cuh"
 #include "ttt.h"
 
 using namespace ttt;
@@ -89,8 +90,14 @@ struct Ws {
   float* rk;           // [T][H]
   float* rq;           // [T][H]
   __half* wsh16;       // [3][H*m][d] fp16: W1, W3, W2^T (gradient kernel)
-  __half* kh16;        // [T][H*d] fp16 K^ (gradient kernel operand)
-  __half* vh16;        // [T][H*d] fp16 V
+  float* etapart;      // [ETA_PARTS] block maxima of |eta| (value scale s of V')
+  __half* kh16;        // [T][H*d] fp16 K^ (gradient operand)
+  __half* vh16;        // [T][H*d] fp16 V' = -s eta v
+  // wide-head path only (d, m multiples of 256): fp16 intermediates [T][H*m]
+  __half* z16;         // Z = V' W2 (scaled dL/du)
+  __half* dh1;         // dL/dh1 (the apply's P, bf16, reuses this buffer)
+  __half* dh3;         // dL/dh3
+  __half* u16;         // u
   size_t total;
   int s_max;
 };
@@ -105,8 +112,13 @@ int split_cap(const ttt_dims& d, ttt_dtype dt) {
 
 bool dims_ok(const ttt_dims& d) { return d.heads >= 1 && d.d >= 1 && d.m >= 1 && d.heads <= 4096; }
 
+// bf16 heads of width d, m multiples of 256 (e.g. d = 1024, m = 2048) run the
+// wide-head path of kernels_wide.cuh; d in {128, 192} the fused kernels.
+bool wide_dims(const ttt_dims& d) { return d.d >= 256 && d.d % 256 == 0 && d.m % 256 == 0 && d.d <= 8192 && d.m <= 16384; }
+
 int dims_supported(const ttt_dims& d, ttt_dtype dt) {
-  if (dt == TTT_BF16) return (d.d == 128 || d.d == 192) && d.m % TC_MS == 0 ? TTT_OK : TTT_ERR_UNSUPPORTED;
+  if (dt == TTT_BF16)
+    return ((d.d == 128 || d.d == 192) && d.m % TC_MS == 0) || wide_dims(d) ? TTT_OK : TTT_ERR_UNSUPPORTED;
   if (dt == TTT_FP32) return (d.d <= 256 && d.d % 4 == 0 && d.m % F32_MS == 0) ? TTT_OK : TTT_ERR_UNSUPPORTED;
   return TTT_ERR_INVALID;
 }
@@ -141,8 +153,15 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_rq = take((size_t)std::max<int64_t>(T, 1) * H * 4);
   const bool tc = dt == TTT_BF16;
   const size_t o_wsh16 = tc ? take(3 * n * 2) : 0;
-  const size_t o_kh = tc ? take((size_t)std::max<int64_t>(T, 1) * H * d * 2) : 0;
-  const size_t o_vh = tc ? take((size_t)std::max<int64_t>(T, 1) * H * d * 2) : 0;
+  const size_t o_etap = tc ? take(ETA_PARTS * 4) : 0;
+  const bool wide = tc && wide_dims(dm);
+  const size_t tokd = (size_t)std::max<int64_t>(T, 1) * H * d * 2, tokm = (size_t)std::max<int64_t>(T, 1) * H * m * 2;
+  const size_t o_kh = tc ? take(tokd) : 0;
+  const size_t o_vh = tc ? take(tokd) : 0;
+  const size_t o_z = wide ? take(tokm) : 0;
+  const size_t o_dh1 = wide ? take(tokm) : 0;
+  const size_t o_dh3 = wide ? take(tokm) : 0;
+  const size_t o_u = wide ? take(tokm) : 0;
   w.total = off;
   uint8_t* b = static_cast<uint8_t*>(base);
   if (b) {
@@ -164,8 +183,15 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
     w.rq = reinterpret_cast<float*>(b + o_rq);
     if (tc) {
       w.wsh16 = reinterpret_cast<__half*>(b + o_wsh16);
+      w.etapart = reinterpret_cast<float*>(b + o_etap);
       w.kh16 = reinterpret_cast<__half*>(b + o_kh);
       w.vh16 = reinterpret_cast<__half*>(b + o_vh);
+      if (wide) {
+        w.z16 = reinterpret_cast<__half*>(b + o_z);
+        w.dh1 = reinterpret_cast<__half*>(b + o_dh1);
+        w.dh3 = reinterpret_cast<__half*>(b + o_dh3);
+        w.u16 = reinterpret_cast<__half*>(b + o_u);
+      }
     }
   }
   return w;
@@ -407,14 +433,25 @@ int launch_shadow(const ttt_weights& W, const Ws& w, const ttt_dims& d, cudaStre
   return TTT_OK;
 }
 
-// fp16 gradient operands K^ and V' = -2^8 eta v (dense [T][H*d]) from the caller's bf16 K, V
-int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta, int64_t T,
-                   const ttt_dims& d, int l2norm, const Ws& w, cudaStream_t s) {
-  if (T == 0) return TTT_OK;
-  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 16));
+// block maxima of |eta| over T x H values -> w.etapart (they fix the value scale s)
+int launch_eta_absmax(const float* eta, int64_t T, const ttt_dims& d, const Ws& w, cudaStream_t s) {
+  const int64_t n = T * d.heads;
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ETA_PARTS, (n + 2047) / 2048));
   ProfScope ps(TTT_PROF_NORM, s);
-  k_prep_kv<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, -GRAD_SCALE,
-                                   w.kh16, w.vh16, T, d.heads, d.d, l2norm);
+  k_eta_absmax<<<blocks, 512, 0, s>>>(eta, n, w.etapart, ETA_PARTS);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+// fp16 gradient operands of T tokens (dense [T][H*d], written at kh, vh) from the
+// caller's bf16 K, V: K^ and V' = -s eta v with the value scale s of w.etapart.
+int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta, int64_t T,
+                   const ttt_dims& d, int l2norm, const Ws& w, __half* kh, __half* vh, cudaStream_t s) {
+  if (T == 0) return TTT_OK;
+  ProfScope ps(TTT_PROF_NORM, s);
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 16));
+  k_prep_kv<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, w.etapart, kh,
+                                   vh, T, d.heads, d.d, l2norm);
   TTT_LAUNCHED();
   return TTT_OK;
 }
@@ -428,13 +465,15 @@ struct UpdOperands {
 };
 
 // Operands of the gradient kernels for T tokens: fp16 K^/V' copies in bf16 mode
-// (V' carries the per-token weights eta), the caller's K/V plus per-token inverse
-// norms in fp32 mode.
+// (V' carries the per-token weights eta and the value scale s; w.etapart the
+// |eta| maxima that fix s), the caller's K/V plus per-token inverse norms in
+// fp32 mode.
 int prepare_update_operands(const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta, int64_t T,
                             const ttt_dims& d, ttt_dtype dt, int l2norm, const Ws& w, cudaStream_t s,
                             UpdOperands* op) {
   if (dt == TTT_BF16) {
-    TTT_TRY(launch_prep_kv(K, ldk, V, ldv, eta, T, d, l2norm, w, s));
+    if (T > 0) TTT_TRY(launch_eta_absmax(eta, T, d, w, s));
+    TTT_TRY(launch_prep_kv(K, ldk, V, ldv, eta, T, d, l2norm, w, w.kh16, w.vh16, s));
     const int64_t hd = (int64_t)d.heads * d.d;
     *op = {w.kh16, hd, w.vh16, hd, nullptr};
     return TTT_OK;
@@ -447,17 +486,201 @@ int prepare_update_operands(const void* K, int64_t ldk, const void* V, int64_t l
   return TTT_OK;
 }
 
+// ---- wide-head path (kernels_wide.cuh)
+
+// One persistent launch of k_wgemm on 2-SM pairs: n_items output tiles, one pair per
+// two SMs (or fewer pairs when there are fewer tiles).
+template <int EPI, bool AMN, bool BMN>
+int launch_wgemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b0,
+                 const CUtensorMap& b1, const WgArgs& args, int n_items, const Ws& w, cudaStream_t s) {
+  if (n_items <= 0) return TTT_OK;
+  auto k = k_wgemm<EPI, AMN, BMN>;
+  TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, WgLayout::ALLOC));
+  const int npairs = std::max(1, std::min(n_items, sm_count() / 2));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * npairs);
+  cfg.blockDim = dim3(WG_THREADS);
+  cfg.dynamicSmemBytes = WgLayout::ALLOC;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  TTT_CHECK(cudaLaunchKernelEx(&cfg, k, a0, a1, a2, b0, b1, args, n_items, w.status, wait_timeout_ns()));
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+WgArgs wg_args() {
+  WgArgs a{};
+  a.mt = a.nt = a.nt2 = a.nmat = a.heads = a.S = 1;
+  return a;
+}
+
+// K-major operand map: rows of `cols` elements (2 bytes each), 64 x 128 boxes.
+bool tmap_k(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, uint64_t ld, bool f16) {
+  return tmap_bf16(tm, base, cols, rows, ld * 2, 64, 128,
+                   f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+// MN-major operand map over token rows: 64 x 64 boxes (64 columns of 64 tokens).
+bool tmap_mn(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows) {
+  return tmap_bf16(tm, base, cols, rows, cols * 2, 64, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+}
+
+// Gradient of the wide path from the prepared fp16 operands K^, V' ([T][H*d]):
+// Z, dH1/dH3/u, then split-K weight gradients (partials scaled by 1/s) and the
+// fixed-order reduction into G.
+int run_grad_wide(const void* K, const void* V, int64_t T, const ttt_dims& d, const Ws& w, float* G,
+                  cudaStream_t s, bool accumulate) {
+  const int H = d.heads, dd = d.d, mm = d.m;
+  const int64_t n = (int64_t)H * mm * dd;
+  const uint64_t hd = (uint64_t)H * dd, hm = (uint64_t)H * mm;
+  CUtensorMap tKh, tVh, tW, tKm, tVm, tD1, tD3, tU;
+  if (!tmap_k(&tKh, K, hd, (uint64_t)T, hd, true) || !tmap_k(&tVh, V, hd, (uint64_t)T, hd, true) ||
+      !tmap_k(&tW, w.wsh16, (uint64_t)dd, 3ull * H * mm, (uint64_t)dd, true) ||
+      !tmap_mn(&tKm, K, hd, (uint64_t)T) || !tmap_mn(&tVm, V, hd, (uint64_t)T) ||
+      !tmap_mn(&tD1, w.dh1, hm, (uint64_t)T) || !tmap_mn(&tD3, w.dh3, hm, (uint64_t)T) ||
+      !tmap_mn(&tU, w.u16, hm, (uint64_t)T))
+    return TTT_ERR_CUDA;
+  const int mt = (int)((T + 255) / 256);
+  ProfScope ps(TTT_PROF_GRAD, s);
+  {  // Z = V' W2 (B rows: the W2^T block of the fp16 weight copy)
+    WgArgs a = wg_args();
+    a.M = (int)T;
+    a.mt = mt;
+    a.nt = mm / 256;
+    a.heads = H;
+    a.kblocks = dd / 64;
+    a.a_head = dd;
+    a.b_row0 = 2 * H * mm;
+    a.b_head = mm;
+    a.out_head = mm;
+    a.out = w.z16;
+    a.ldo = (int64_t)hm;
+    a.idesc = idesc_f16(256, 256, false, false);
+    TTT_TRY((launch_wgemm<WG_STORE16, false, false>(tVh, tVh, tVh, tW, tW, a, mt * a.nt * H, w, s)));
+  }
+  {  // [H1 | H3] = K^ [W1; W3]^T, 128 m columns per tile -> dH1, dH3, u
+    WgArgs a = wg_args();
+    a.M = (int)T;
+    a.mt = mt;
+    a.nt = mm / 128;
+    a.heads = H;
+    a.kblocks = dd / 64;
+    a.a_head = dd;
+    a.b_row0 = 0;
+    a.b_head = mm;
+    a.b_row1 = H * mm;
+    a.m = mm;
+    a.d = dd;
+    a.out = w.dh1;
+    a.out2 = w.dh3;
+    a.out3 = w.u16;
+    a.aux = w.z16;
+    a.ldo = a.ldaux = (int64_t)hm;
+    a.idesc = idesc_f16(256, 256, false, false);
+    TTT_TRY((launch_wgemm<WG_SWIGLU_BWD, false, false>(tKh, tKh, tKh, tW, tW, a, mt * a.nt * H, w, s)));
+  }
+  int S = 1;
+  {  // g1 = dH1^T K^, g3 = dH3^T K^, g2 = V'^T u: token-split partials
+    WgArgs a = wg_args();
+    const int tiles = (mm / 256) * (dd / 256);
+    const int kblocks = (int)((T + 63) / 64);
+    S = std::max(1, std::min({w.s_max, kblocks, (sm_count() / 2 * 4 + 3 * H * tiles - 1) / (3 * H * tiles)}));
+    a.M = std::max(mm, dd);
+    a.mt = mm / 256;
+    a.nt = dd / 256;
+    a.nt2 = mm / 256;
+    a.nmat = 3;
+    a.heads = H;
+    a.S = S;
+    a.kblocks = kblocks;
+    a.a_head = mm;
+    a.b_head = dd;
+    a.mat2_a_head = dd;
+    a.mat2_b_head = mm;
+    a.m = mm;
+    a.d = dd;
+    a.out = w.partial;
+    a.eta_part = w.etapart;
+    a.idesc = idesc_f16(256, 256, true, true);
+    TTT_TRY((launch_wgemm<WG_PARTIAL, true, true>(tD1, tD3, tVm, tKm, tU, a, S * 3 * H * tiles, w, s)));
+  }
+  k_reduce_splits<<<grid1d(3 * n / 4, 256), 256, 0, s>>>(w.partial, S, 3 * n, G, accumulate ? 1 : 0, w.status);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
+
+// Apply of the wide path: P = SiLU(r Q W1^T) o (r Q W3^T) (bf16, in the dH1 buffer), O = P W2^T.
+int run_apply_wide(const void* Q, int64_t ldq, void* O, int64_t ldo, int qnorm, float* rq_buf, int64_t T,
+                   const ttt_dims& d, const Ws& w, cudaStream_t s) {
+  const int H = d.heads, dd = d.d, mm = d.m;
+  const uint64_t hd = (uint64_t)H * dd, hm = (uint64_t)H * mm;
+  if (qnorm) TTT_TRY(launch_rownorm_any(Q, ldq, T, d, TTT_BF16, rq_buf, s));
+  __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(w.dh1);
+  CUtensorMap tQ, tW, tP, tW2;
+  if (!tmap_k(&tQ, Q, hd, (uint64_t)T, (uint64_t)ldq, false) ||
+      !tmap_k(&tW, w.wsh, (uint64_t)dd, 3ull * H * mm, (uint64_t)dd, false) ||
+      !tmap_k(&tP, P, hm, (uint64_t)T, hm, false) || !tmap_k(&tW2, w.w2b, (uint64_t)mm, hd, (uint64_t)mm, false))
+    return TTT_ERR_CUDA;
+  const int mt = (int)((T + 255) / 256);
+  ProfScope ps(TTT_PROF_APPLY, s);
+  {
+    WgArgs a = wg_args();
+    a.M = (int)T;
+    a.mt = mt;
+    a.nt = mm / 128;
+    a.heads = H;
+    a.kblocks = dd / 64;
+    a.a_head = dd;
+    a.b_row0 = 0;
+    a.b_head = mm;
+    a.b_row1 = H * mm;
+    a.m = mm;
+    a.d = dd;
+    a.out = P;
+    a.ldo = (int64_t)hm;
+    a.rvec = qnorm ? rq_buf : nullptr;
+    a.idesc = idesc_bf16(256, 256, false, false);
+    TTT_TRY((launch_wgemm<WG_SWIGLU_FWD, false, false>(tQ, tQ, tQ, tW, tW, a, mt * a.nt * H, w, s)));
+  }
+  {
+    WgArgs a = wg_args();
+    a.M = (int)T;
+    a.mt = mt;
+    a.nt = dd / 256;
+    a.heads = H;
+    a.kblocks = mm / 64;
+    a.a_head = mm;
+    a.b_row0 = 0;
+    a.b_head = dd;
+    a.out_head = dd;
+    a.out = O;
+    a.ldo = ldo;
+    a.idesc = idesc_bf16(256, 256, false, false);
+    TTT_TRY((launch_wgemm<WG_STORE_BF16, false, false>(tP, tP, tP, tW2, tW2, a, mt * a.nt * H, w, s)));
+  }
+  return TTT_OK;
+}
+
 // gradient over T tokens -> G (fp32, [3][H*m*d]); shadow of W must be current.
-// bf16 mode: K, V are the fp16 operands written by launch_prep_kv (ld = H*d, K^ normalised).
-// accumulate = true adds the gradient to G instead of overwriting it.
+// bf16 mode: K, V are the fp16 operands K^, V' of prepare_update_operands (ld = H*d)
+// and w.etapart holds the |eta| maxima of these T tokens; qk is not read there
+// (K^ is already normalised).  accumulate = true adds the gradient to G instead
+// of overwriting it.
 int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta,
-             const float* rk, int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, float* G, cudaStream_t s,
-             bool accumulate = false) {
+             const float* rk, int qk, int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, float* G,
+             cudaStream_t s, bool accumulate = false) {
   const int64_t n = (int64_t)d.heads * d.m * d.d;
   if (T == 0) {
     if (!accumulate) TTT_CHECK(cudaMemsetAsync(G, 0, 3 * n * sizeof(float), s));
     return TTT_OK;
   }
+  (void)qk;
+  if (dt == TTT_BF16 && wide_dims(d)) return run_grad_wide(K, V, T, d, w, G, s, accumulate);
   int S = 1;
   if (dt == TTT_BF16) {
     const int tiles = (int)((T + TC_TILE - 1) / TC_TILE);
@@ -477,13 +700,13 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
     if (d.d == 192) {
       auto k = k_update_grad_tc<192>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<192>::ALLOC));
-      k<<<grid, UPD_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, w.partial, T, d.heads, d.m,
-                                                          tiles, S, w.status, wait_timeout_ns());
+      k<<<grid, UPD_THREADS, UpdLayout<192>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, w.etapart, w.partial, T, d.heads,
+                                                          d.m, tiles, S, w.status, wait_timeout_ns());
     } else {
       auto k = k_update_grad_tc<128>;
       TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, UpdLayout<128>::ALLOC));
-      k<<<grid, UPD_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, w.partial, T, d.heads, d.m,
-                                                          tiles, S, w.status, wait_timeout_ns());
+      k<<<grid, UPD_THREADS, UpdLayout<128>::ALLOC, s>>>(tK, tV, tKb, tVb, tW, w.etapart, w.partial, T, d.heads,
+                                                          d.m, tiles, S, w.status, wait_timeout_ns());
     }
     TTT_LAUNCHED();
   } else {
@@ -499,7 +722,7 @@ int run_grad(const ttt_weights& W, const void* K, int64_t ldk, const void* V, in
     TTT_LAUNCHED();
   }
   ProfScope ps(TTT_PROF_REDUCE, s);
-  k_reduce_splits<<<grid1d(3 * n / 4, 256), 256, 0, s>>>(w.partial, S, 3 * n, G, accumulate ? 1 : 0);
+  k_reduce_splits<<<grid1d(3 * n / 4, 256), 256, 0, s>>>(w.partial, S, 3 * n, G, accumulate ? 1 : 0, w.status);
   TTT_LAUNCHED();
   return TTT_OK;
 }
@@ -513,7 +736,7 @@ int run_step_update(const ttt_weights& W, const float* Dw, const float* Dt, cons
   TTT_TRY(launch_pdl(k_step_partials, dim3(nb, NORM_PARTS), dim3(256), 0, s, W.W1, W.W3, W.W2, Dw, Dt, H, dd, mm,
                      ns.lr, w.stepn));
   return launch_pdl(k_step_apply, dim3(grid1d(n / 4, 256) / nb + 1, nb), dim3(256), 0, s, W.W1, W.W3, W.W2, Dw, Dt, H,
-                    dd, mm, ns.lr, ns.renorm, (const float*)w.stepn);
+                    dd, mm, ns.lr, ns.renorm, (const float*)w.stepn, (const unsigned int*)w.status);
 }
 
 // C = alpha A B + beta Cin on the tensor cores (split bf16 parts); see kernels_nsmma.cuh
@@ -542,7 +765,9 @@ int launch_mm3_r(int r, int K, int ksplit, int nsplit, int batch, const float* A
   if (r <= 192)
     return launch_mm3<192, BK>(r, r, K, ksplit, nsplit, batch, A, lda, sA, B, ldb, sB, C, r, sC, sCsplit, Cin, alpha,
                                beta, w, s);
-  return TTT_ERR_UNSUPPORTED;
+  // wide heads: 128 x 128 tiles over the r x r product
+  return launch_mm3<128, BK>(r, r, K, ksplit, nsplit, batch, A, lda, sA, B, ldb, sB, C, r, sC, sCsplit, Cin, alpha,
+                             beta, w, s);
 }
 
 // Newton-Schulz iterations of the bf16 path on the tensor cores: X (r x c) -> X
@@ -680,6 +905,7 @@ int run_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, const t
 int run_apply(const ttt_weights& W, const void* Q, int64_t ldq, void* O, int64_t ldo, int qnorm, float* rq_buf,
               int64_t T, const ttt_dims& d, ttt_dtype dt, const Ws& w, cudaStream_t s) {
   if (T == 0) return TTT_OK;
+  if (dt == TTT_BF16 && wide_dims(d)) return run_apply_wide(Q, ldq, O, ldo, qnorm, rq_buf, T, d, w, s);
   if (dt == TTT_BF16) {
     const int pair_tiles = (int)((T + 2 * TC_TILE - 1) / (2 * TC_TILE));
     const int n_items = pair_tiles * d.heads;
@@ -834,7 +1060,8 @@ int ttt_poll_status(const void* ws, void* stream) {
   TTT_CHECK(cudaStreamSynchronize((cudaStream_t)stream));
   unsigned int v = 0;
   TTT_CHECK(cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost));
-  return v == DEV_OK ? TTT_OK : TTT_ERR_TIMEOUT;
+  if (v == DEV_OK) return TTT_OK;
+  return v == DEV_RANGE ? TTT_ERR_RANGE : TTT_ERR_TIMEOUT;
 }
 
 int ttt_l2norm(void* X, int64_t T, ttt_dims dims, int64_t ld, ttt_dtype dtype, void* stream) {
@@ -878,7 +1105,7 @@ int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int6
   UpdOperands op;
   TTT_TRY(prepare_update_operands(K, ldk, V, ldv, eta, T, dims, dtype, io->qk_l2norm, w, s, &op));
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
-  return run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, T, dims, dtype, w, G, s);
+  return run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, io->qk_l2norm, T, dims, dtype, w, G, s);
 }
 
 int ttt_step(ttt_weights W, const float* G, const ttt_ns_cfg* ns, ttt_dims dims, ttt_dtype dtype, void* ws,
@@ -910,7 +1137,7 @@ int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, in
   TTT_TRY(prepare_update_operands(K, ldk, V, ldv, eta, T, dims, dtype, io->qk_l2norm, w, s, &op));
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
   for (int st = 0; st < steps; ++st) {
-    TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, T, dims, dtype, w, w.G, s));
+    TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, io->qk_l2norm, T, dims, dtype, w, w.G, s));
     TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
   }
   return TTT_OK;
@@ -943,6 +1170,8 @@ int ttt_apply_noalloc(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims
   TTT_TRY(check_tokens(Q, ldq, dims, dtype, T));
   TTT_TRY(check_tokens(O, ldo, dims, dtype, T));
   if (T > 0 && Q == O) return TTT_ERR_INVALID;
+  // the wide-head apply needs a per-token intermediate that this fixed scratch does not hold
+  if (dtype == TTT_BF16 && wide_dims(dims)) return TTT_ERR_UNSUPPORTED;
   // scratch plan: [status 256 B | W1,W3,W2^T bf16 | W2 bf16 | per-token inverse norms of one token chunk]
   const size_t n = (size_t)dims.heads * dims.m * dims.d;
   const size_t fixed = 256 + up256(3 * n * 2) + up256(n * 2);
@@ -1004,7 +1233,7 @@ int ttt_chunked(ttt_weights W, const void* Q, const void* K, const void* V, cons
     TTT_TRY(prepare_update_operands(k, ldk, v, ldv, e, tc, dims, dtype, io->qk_l2norm, w, s, &op));
     if (order == 0) TTT_TRY(run_apply(W, q, ldq, o, ldo, io->qk_l2norm, w.rq, tc, dims, dtype, w, s));
     for (int st = 0; st < steps; ++st) {
-      TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, e, op.rk, tc, dims, dtype, w, w.G, s));
+      TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, e, op.rk, io->qk_l2norm, tc, dims, dtype, w, w.G, s));
       TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
     }
     if (order == 1) TTT_TRY(run_apply(W, q, ldq, o, ldo, io->qk_l2norm, w.rq, tc, dims, dtype, w, s));
@@ -1077,13 +1306,20 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
     return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, P->h2d);
   };
   auto body = [&]() -> int {
+    // bidirectional: all of eta first (4 H bytes per token), so the value scale of
+    // the whole update is known before the first block's operands are prepared
+    if (chunk == 0)
+      TTT_CHECK(up(reinterpret_cast<uint8_t*>(dEta), reinterpret_cast<const uint8_t*>(hEta),
+                   (size_t)T * dims.heads * 4));
     for (int64_t b = 0; b < nb; ++b) {
       const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
       TTT_CHECK(up(dK + t0 * row, cK + t0 * row, tb * row));
       TTT_CHECK(up(dV + t0 * row, cV + t0 * row, tb * row));
-      TTT_CHECK(up(reinterpret_cast<uint8_t*>(dEta + t0 * dims.heads),
-                   reinterpret_cast<const uint8_t*>(hEta + t0 * dims.heads), (size_t)tb * dims.heads * 4));
-      if (chunk > 0) TTT_CHECK(up(dQ + t0 * row, cQ + t0 * row, tb * row));
+      if (chunk > 0) {
+        TTT_CHECK(up(reinterpret_cast<uint8_t*>(dEta + t0 * dims.heads),
+                     reinterpret_cast<const uint8_t*>(hEta + t0 * dims.heads), (size_t)tb * dims.heads * 4));
+        TTT_CHECK(up(dQ + t0 * row, cQ + t0 * row, tb * row));
+      }
       TTT_CHECK(cudaEventRecord(ev_in[b], P->h2d));
     }
     if (chunk == 0)
@@ -1124,7 +1360,7 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
                                           io->qk_l2norm, w, s, &op));
           for (int st = 0; st < steps; ++st) {
             TTT_TRY(
-                run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s));
+                run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, io->qk_l2norm, tb, dims, dtype, w, w.G, s));
             TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
           }
         }
@@ -1133,24 +1369,30 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
       return TTT_OK;
     }
     if (steps > 0) {
-      // first step: preparation and gradient block by block as the blocks land
+      // first step: preparation and gradient block by block as the blocks land; the
+      // bf16 operands of all blocks share the value scale of the whole eta
+      if (dtype == TTT_BF16) {
+        TTT_CHECK(cudaStreamWaitEvent(s, ev_in[0], 0));  // eta (copied first) is on the device
+        TTT_TRY(launch_eta_absmax(dEta, T, dims, w, s));
+      }
       for (int64_t b = 0; b < nb; ++b) {
         const int64_t t0 = b * bt, tb = std::min(bt, T - t0);
         TTT_CHECK(cudaStreamWaitEvent(s, ev_in[b], 0));
         const uint8_t* v = vsrc(t0, tb);
         if (!v) return TTT_ERR_CUDA;
-        Ws wb = w;  // per-token operand buffers shifted to the block
-        if (dtype == TTT_BF16) {
-          wb.kh16 = w.kh16 + t0 * hd;
-          wb.vh16 = w.vh16 + t0 * hd;
-        } else {
-          wb.rk = w.rk + t0 * dims.heads;
-        }
         UpdOperands op;
-        TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, dEta + t0 * dims.heads, tb, dims, dtype,
-                                        io->qk_l2norm, wb, s, &op));
-        TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, tb, dims, dtype, w, w.G, s,
-                         b > 0));
+        if (dtype == TTT_BF16) {
+          TTT_TRY(launch_prep_kv(dK + t0 * row, hd, v, hd, dEta + t0 * dims.heads, tb, dims, io->qk_l2norm, w,
+                                 w.kh16 + t0 * hd, w.vh16 + t0 * hd, s));
+          op = {w.kh16 + t0 * hd, hd, w.vh16 + t0 * hd, hd, nullptr};
+        } else {
+          Ws wb = w;  // the per-token inverse norms shifted to the block
+          wb.rk = w.rk + t0 * dims.heads;
+          TTT_TRY(prepare_update_operands(dK + t0 * row, hd, v, hd, dEta + t0 * dims.heads, tb, dims, dtype,
+                                          io->qk_l2norm, wb, s, &op));
+        }
+        TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, dEta + t0 * dims.heads, op.rk, io->qk_l2norm, tb, dims,
+                         dtype, w, w.G, s, b > 0));
       }
       TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
       // further steps re-read the prepared operands of all T tokens
@@ -1160,7 +1402,7 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
       else
         full = {dK, hd, conv ? dVc : dV, hd, io->qk_l2norm ? w.rk : nullptr};
       for (int st = 1; st < steps; ++st) {
-        TTT_TRY(run_grad(W, full.K, full.ldk, full.V, full.ldv, dEta, full.rk, T, dims, dtype, w, w.G, s));
+        TTT_TRY(run_grad(W, full.K, full.ldk, full.V, full.ldv, dEta, full.rk, io->qk_l2norm, T, dims, dtype, w, w.G, s));
         TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
       }
     }
@@ -1179,6 +1421,56 @@ int ttt_layer_host(ttt_weights W, const void* hQ, const void* hK, const void* hV
   if (rc != TTT_OK) return rc;
   if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess || e4 != cudaSuccess) return TTT_ERR_CUDA;
   return TTT_OK;
+}
+
+size_t ttt_gate_workspace_bytes(int64_t T, int D) {
+  if (T < 0 || D < 256 || D % 256) return 0;
+  return 256 + up256((size_t)D * D * 2) + up256((size_t)std::max<int64_t>(T, 1) * 4);
+}
+
+int ttt_output_gate(const void* Oprime, int64_t ld_in, const float* Wg, void* O, int64_t ld_out, int64_t T, int D,
+                    ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (dtype != TTT_FP32 && dtype != TTT_BF16) return TTT_ERR_INVALID;
+  if (T < 0 || D < 1) return TTT_ERR_INVALID;
+  if (dtype != TTT_BF16 || D % 256 || D < 256 || T > INT32_MAX) return TTT_ERR_UNSUPPORTED;
+  if (ld_in == 0) ld_in = D;
+  if (ld_out == 0) ld_out = D;
+  if (ld_in < D || ld_out < D) return TTT_ERR_INVALID;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTT_ERR_WORKSPACE;
+  if (ws_bytes < ttt_gate_workspace_bytes(T, D)) return TTT_ERR_WORKSPACE;
+  if (T == 0) return TTT_OK;
+  if (!Oprime || !Wg || !O || Oprime == O) return TTT_ERR_INVALID;
+  if (!aligned16(Oprime) || !aligned16(O) || !aligned16(Wg) || (ld_in * 2) % 16 || (ld_out * 2) % 16)
+    return TTT_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  Ws w{};
+  w.status = reinterpret_cast<unsigned int*>(b);
+  __nv_bfloat16* wg16 = reinterpret_cast<__nv_bfloat16*>(b + 256);
+  float* rinv = reinterpret_cast<float*>(b + 256 + up256((size_t)D * D * 2));
+  const int64_t nn = (int64_t)D * D;
+  ProfScope ps(TTT_PROF_APPLY, s);
+  k_cast_bf16<<<grid1d(nn / 4, 256), 256, 0, s>>>(Wg, wg16, nn);
+  TTT_LAUNCHED();
+  k_rms_rows<<<(int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 16)), 256, 0,
+               s>>>((const __nv_bfloat16*)Oprime, ld_in, T, D, 1e-6f, rinv);
+  TTT_LAUNCHED();
+  CUtensorMap tA, tB;
+  if (!tmap_k(&tA, Oprime, (uint64_t)D, (uint64_t)T, (uint64_t)ld_in, false) ||
+      !tmap_k(&tB, wg16, (uint64_t)D, (uint64_t)D, (uint64_t)D, false))
+    return TTT_ERR_CUDA;
+  WgArgs a = wg_args();
+  a.M = (int)T;
+  a.mt = (int)((T + 255) / 256);
+  a.nt = D / 256;
+  a.kblocks = D / 64;
+  a.out = O;
+  a.ldo = ld_out;
+  a.aux = Oprime;
+  a.ldaux = ld_in;
+  a.rvec = rinv;
+  a.idesc = idesc_bf16(256, 256, false, false);
+  return launch_wgemm<WG_GATE, false, false>(tA, tA, tA, tB, tB, a, a.mt * a.nt, w, s);
 }
 
 int ttt_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned timeout_us, void* stream) {
@@ -1216,6 +1508,7 @@ const char* ttt_status_string(int status) {
     case TTT_ERR_TIMEOUT: return "device-side wait timed out";
     case TTT_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
     case TTT_ERR_SCRATCH: return "problem too large for the fixed 8 MiB scratch of ttt_apply_noalloc";
+    case TTT_ERR_RANGE: return "gradient not finite: an fp16 operand of the tensor-core update was out of range";
     default: return "unknown status";
   }
 }

@@ -28,6 +28,10 @@ Workloads (the pages give shapes, not data; these stand in for their datasets):
                 frame by frame (chunk = one frame of 37x37 + 5 tokens, 750
                 chunks), each frame's outputs from the weights after its own
                 update (order 1).
+* ``zipmap1024`` ZipMap's own head shape: one head with token dim d = 1024
+                and hidden m = 2048 (state 6 d^2), the zipmap token recipe, and
+                the gated output o = RMSNorm(o') SiLU(W_g o') with a random
+                W_g ~ N(0, 1/D).
 """
 from __future__ import annotations
 
@@ -39,7 +43,7 @@ import torch
 BLOCK = 1 << 14
 
 # tensor ids used to derive independent streams
-TID_Q, TID_K, TID_V, TID_ETA, TID_ETA_X, TID_ETA_W, TID_W, TID_TAPS = 1, 2, 3, 4, 5, 6, 7, 8
+TID_Q, TID_K, TID_V, TID_ETA, TID_ETA_X, TID_ETA_W, TID_W, TID_TAPS, TID_GATE = 1, 2, 3, 4, 5, 6, 7, 8, 9
 
 _MASK64 = (1 << 64) - 1
 
@@ -116,6 +120,11 @@ def init_weights(seed: int, H: int, d: int, m: int):
     return W1.contiguous(), W3.contiguous(), W2.contiguous()
 
 
+def gate_weight(seed: int, D: int) -> torch.Tensor:
+    """Output-gate weight W_g ~ N(0, 1/D), fp32 [D, D] (row j produces gate j)."""
+    return normal_rows(seed, TID_GATE, 0, D, D, torch.float32, std=1.0 / math.sqrt(D)).contiguous()
+
+
 def conv_taps(seed: int, C: int) -> torch.Tensor:
     """Depthwise 3x3 taps ~ N(0, 1/9), fp32 [C, 3, 3]."""
     return normal_rows(seed, TID_TAPS, 0, C, 9, torch.float32, std=1.0 / 3.0).reshape(C, 3, 3).contiguous()
@@ -139,6 +148,7 @@ class Workload:
     chunk: int = 0              # 0: one bidirectional chunk
     order: int = 0              # chunked: 0 apply with the carried W, then update; 1 update, then apply
     query_tokens: int = 0       # >0: apply on separate query tokens instead of Q of the context
+    gate: bool = False          # gated output o = RMSNorm(o') SiLU(W_g o') after the apply
     ns_iters: int = 5
     ns_a: float = 3.4445
     ns_b: float = -4.7750
@@ -168,7 +178,9 @@ class Workload:
         return 12.0 * self.heads * self.d * self.m * self.tokens * self.steps
 
     def apply_flops(self) -> float:
-        return 6.0 * self.heads * self.d * self.m * self.apply_tokens
+        """6*H*d*m flops per query token, plus the gate's 2*D^2 when it is on."""
+        gate = 2.0 * self.model_dim * self.model_dim * self.apply_tokens if self.gate else 0.0
+        return 6.0 * self.heads * self.d * self.m * self.apply_tokens + gate
 
     def ns_flops(self) -> float:
         """Newton-Schulz flops per layer: 3H matrices, per iteration 2 r^2 c + 2 r^3 + 2 r^2 c."""
@@ -198,6 +210,8 @@ WORKLOADS = {
                       chunk=128 * 1024),
     "stream": Workload("stream", 1005, heads=4, d=192, m=768, frames=750, grid_h=37, grid_w=37,
                        special=5, eta_kind="linear", chunk=37 * 37 + 5, order=1),
+    "zipmap1024": Workload("zipmap1024", 1006, heads=1, d=1024, m=2048, frames=750, grid_h=37, grid_w=37,
+                           special=5, eta_kind="linear", gate=True),
 }
 
 
@@ -229,3 +243,6 @@ class Inputs:
 
     def taps(self):
         return conv_taps(self.cfg.seed, self.cfg.model_dim)
+
+    def gate_weight(self):
+        return gate_weight(self.cfg.seed, self.cfg.model_dim)

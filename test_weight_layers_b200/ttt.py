@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libttt.so")
 
 TTT_OK, TTT_ERR_INVALID, TTT_ERR_UNSUPPORTED, TTT_ERR_WORKSPACE = 0, -1, -2, -3
 TTT_ERR_CUDA, TTT_ERR_TIMEOUT, TTT_ERR_ALIGN, TTT_ERR_SCRATCH = -4, -5, -6, -7
+TTT_ERR_RANGE = -8
 TTT_FP32, TTT_BF16 = 0, 1
 
 
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "ttt_host_buffer_bytes": (SZ, [Dims, I64, I, I]),
             "ttt_layer_host": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), P, I, I, Dims,
                                    ctypes.POINTER(IOCfg), I, P, SZ, P, SZ, P]),
+            "ttt_gate_workspace_bytes": (SZ, [I64, I]),
+            "ttt_output_gate": (I, [P, I64, P, P, I64, I64, I, I, P, SZ, P]),
             "ttt_status_string": (ctypes.c_char_p, [I]),
             "ttt_compiled_arch": (I, []),
             "ttt_kernel_binary_version": (I, [ctypes.POINTER(I)]),
@@ -185,6 +188,19 @@ def ttt_apply_noalloc(W: Weights, Q, O, T, dm: Dims, io: IOCfg, stream=None):
     """ttt_apply without a workspace: the library uses its own fixed 8 MiB device array as scratch."""
     _check("ttt_apply_noalloc", lib().ttt_apply_noalloc(W, _ptr(Q), _ptr(O), T, dm, ctypes.byref(io),
                                                         dtype_code(Q.dtype), _stream(stream)))
+
+
+def gate_workspace(T: int, D: int, device="cuda") -> torch.Tensor:
+    n = int(lib().ttt_gate_workspace_bytes(T, D))
+    if n == 0:
+        raise TTTError("ttt_gate_workspace_bytes", TTT_ERR_UNSUPPORTED, "D must be a positive multiple of 256")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def ttt_output_gate(Oprime, Wg, O, T, D, ws, ld_in=0, ld_out=0, stream=None):
+    """O = RMSNorm(O') * SiLU(O' W_g^T) per token (bf16 O', O; fp32 W_g [D][D])."""
+    _check("ttt_output_gate", lib().ttt_output_gate(_ptr(Oprime), ld_in, _ptr(Wg), _ptr(O), ld_out, T, D,
+                                                    dtype_code(Oprime.dtype), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def ttt_chunked(W: Weights, Q, K, V, eta, O, T, chunk, order, steps, ns: NSCfg, dm: Dims, io: IOCfg, ws, stream=None):

@@ -134,3 +134,35 @@ def test_layer_host_validation(lib):
     assert _call_layer_host(lib, d, T.TTT_BF16, T_, 0, need_dbc, need_ws, taps=FAKE, gh=7, gw=7) == T.TTT_ERR_INVALID
     assert _call_layer_host(lib, d, T.TTT_BF16, T_, 100, need_dbc, need_ws, taps=FAKE, gh=4, gw=4) \
         == T.TTT_ERR_INVALID
+
+
+def test_output_gate_validation(lib):
+    D, T_ = 1024, 300
+    need = lib.ttt_gate_workspace_bytes(T_, D)
+    assert need >= D * D * 2 + T_ * 4
+    assert lib.ttt_gate_workspace_bytes(T_, 1000) == 0   # D must be a multiple of 256
+    call = lambda Op, Wg, O_, D_, dt, ws_bytes: lib.ttt_output_gate(Op, 0, Wg, O_, 0, T_, D_, dt, FAKE, ws_bytes, None)
+    A, B, C = ctypes.c_void_p(1 << 21), ctypes.c_void_p(1 << 22), ctypes.c_void_p(1 << 23)
+    assert call(A, B, C, D, T.TTT_FP32, need) == T.TTT_ERR_UNSUPPORTED
+    assert call(A, B, C, 768 + 8, T.TTT_BF16, need) == T.TTT_ERR_UNSUPPORTED
+    assert call(A, B, C, D, T.TTT_BF16, need - 1) == T.TTT_ERR_WORKSPACE
+    assert call(A, B, A, D, T.TTT_BF16, need) == T.TTT_ERR_INVALID          # O aliases O'
+    assert call(None, B, C, D, T.TTT_BF16, need) == T.TTT_ERR_INVALID
+    assert call(ctypes.c_void_p((1 << 21) + 2), B, C, D, T.TTT_BF16, need) == T.TTT_ERR_ALIGN
+
+
+def test_wide_head_shapes_are_accepted(lib):
+    # d and m multiples of 256 run the wide-head path in bf16; the workspace holds its
+    # fp16 intermediates (K^, V', Z, dH1, dH3, u: 2 (2 d + 4 m) bytes per token and head)
+    d = T.dims(1, 1024, 2048)
+    small = T.ttt_workspace_bytes(d, 1000, T.TTT_BF16)
+    big = T.ttt_workspace_bytes(d, 2000, T.TTT_BF16)
+    assert big - small >= 1000 * 2 * (2 * 1024 + 4 * 2048)
+    assert _call_update(lib, d, T.TTT_BF16, small - 1, T_=1000) == T.TTT_ERR_WORKSPACE
+    assert _call_update(lib, T.dims(1, 1024, 2000), T.TTT_BF16, 1 << 40) == T.TTT_ERR_UNSUPPORTED
+    assert _call_update(lib, T.dims(1, 1024, 2048), T.TTT_FP32, 1 << 40) == T.TTT_ERR_UNSUPPORTED
+    # the no-allocation apply has no room for the wide path's per-token intermediate
+    W = T.Weights(1 << 20, 1 << 21, 1 << 22)
+    rc = lib.ttt_apply_noalloc(W, FAKE, ctypes.c_void_p(1 << 23), 10, T.dims(1, 256, 256),
+                               ctypes.byref(T.io_cfg()), T.TTT_BF16, None)
+    assert rc == T.TTT_ERR_UNSUPPORTED
