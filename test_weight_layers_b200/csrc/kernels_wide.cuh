@@ -49,7 +49,8 @@ enum WgEpi : int {
   WG_PARTIAL = 2,      // fp32 split-K partial = acc * scale
   WG_SWIGLU_FWD = 3,   // acc = [H1 | H3]: P = SiLU(r H1) o (r H3) (bf16)
   WG_STORE_BF16 = 4,   // C (bf16) = acc
-  WG_GATE = 5          // acc = o' W_g^T: out = o' rinv SiLU(acc) (bf16)
+  WG_GATE = 5,         // acc = o' W_g^T: out = o' rinv SiLU(acc) (bf16)
+  WG_NSOUT = 6         // Newton-Schulz product: C = alpha acc + beta Cin (fp32) and its bf16 hi/lo parts
 };
 
 // Everything a launch needs besides the tensor maps.  Items are
@@ -69,6 +70,9 @@ struct WgArgs {
   int b_row0;     // first row of B (K-major): the weight block inside the fp16/bf16 weight copy
   int b_head;     // per-head row offset of B (K-major) or x offset (MN-major)
   int b_row1;     // SwiGLU products: row of the second half (W3) relative to the first (W1)
+  int a_row_head; // per-matrix row offset of A (K-major; Newton-Schulz batches)
+  int b_y_head;   // per-matrix K-row offset of B (MN-major; Newton-Schulz batches)
+  float alpha, beta;  // WG_NSOUT
   int out_head;   // per-head column offset of a stored output
   int mat2_a_head, mat2_b_head;  // weight gradients: per-head offsets of g2's operands (V', u)
   int m, d;       // head dims (weight gradients, epilogue column offsets)
@@ -225,6 +229,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         wg_krange(a, it.s, k0, k1);
         const CUtensorMap* mA = tA[it.mat];
         const CUtensorMap* mB = tB[it.mat == 2 ? 1 : 0];
+        // Newton-Schulz products run over three K segments of split operands,
+        // hi.hi + hi.lo + lo.hi: A = (hi, hi, lo), B = (hi, lo, hi)
+        const int kseg = EPI == WG_NSOUT ? a.kblocks / 3 : a.kblocks;
         for (int kb = k0; kb < k1; ++kb, ++gs) {
           const int st = gs % WG_STAGES, use = gs / WG_STAGES;
           if (use > 0 && !mbar_wait(bars.empty + st, (use - 1) & 1, g)) { ok = false; break; }
@@ -232,15 +239,23 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
           if (leader) mbar_expect_tx(bars.full + st, 4 * WG_HALF);
           uint8_t* sa = smem + WgLayout::A_OFF + st * WG_HALF;
           uint8_t* sb = smem + WgLayout::B_OFF + st * WG_HALF;
+          int kk = kb * 64;
+          if (EPI == WG_NSOUT) {
+            const int seg = kb / kseg;
+            kk = (kb - seg * kseg) * 64;
+            mA = tA[seg == 2 ? 1 : 0];
+            mB = tB[seg == 1 ? 1 : 0];
+          }
           if constexpr (!AMN) {
             // A rows = output rows (tokens): this CTA's 128 of the tile's 256
-            tma_load_2d_pair(sa, mA, full_l, it.h * a.a_head + kb * 64, it.tm * 256 + (int)rank * 128);
+            tma_load_2d_pair(sa, mA, full_l, it.h * a.a_head + kk,
+                             it.h * a.a_row_head + it.tm * 256 + (int)rank * 128);
           } else {
             // A^T: token rows, 128 output rows as two 64-wide column boxes
             const int ah = it.mat == 2 ? a.mat2_a_head : a.a_head;
             const int x0 = it.h * ah + it.tm * 256 + (int)rank * 128;
-            tma_load_2d_pair(sa, mA, full_l, x0, kb * 64);
-            tma_load_2d_pair(sa + 8192, mA, full_l, x0 + 64, kb * 64);
+            tma_load_2d_pair(sa, mA, full_l, x0, kk);
+            tma_load_2d_pair(sa + 8192, mA, full_l, x0 + 64, kk);
           }
           if constexpr (!BMN) {
             int brow;
@@ -248,12 +263,12 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
               brow = a.b_row0 + it.h * a.b_head + it.tn * 128 + (int)rank * a.b_row1;  // W1 rows | W3 rows
             else
               brow = a.b_row0 + it.h * a.b_head + it.tn * 256 + (int)rank * 128;
-            tma_load_2d_pair(sb, mB, full_l, kb * 64, brow);
+            tma_load_2d_pair(sb, mB, full_l, kk, brow);
           } else {
             const int bh = it.mat == 2 ? a.mat2_b_head : a.b_head;
             const int x0 = it.h * bh + it.tn * 256 + (int)rank * 128;
-            tma_load_2d_pair(sb, mB, full_l, x0, kb * 64);
-            tma_load_2d_pair(sb + 8192, mB, full_l, x0 + 64, kb * 64);
+            tma_load_2d_pair(sb, mB, full_l, x0, it.h * a.b_y_head + kk);
+            tma_load_2d_pair(sb + 8192, mB, full_l, x0 + 64, it.h * a.b_y_head + kk);
           }
         }
       }
@@ -317,130 +332,199 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       float s_;
       value_scale(mx, s_, scale);
     }
+    // SwiGLU backward: this thread's 64 values of Z for an item (Z does not depend on the
+    // MMAs, and its row-strided loads take an L2/HBM round trip)
+    auto z_load = [&](int item, uint4 (&zq)[8]) {
+      if (EPI != WG_SWIGLU_BWD || item >= n_items) return;
+      const WgItem it = wg_item(a, item);
+      const int64_t row = (int64_t)it.tm * 256 + rank * 128 + rloc;
+      if (row >= a.M) return;
+      const __half* zr = static_cast<const __half*>(a.aux) + row * a.ldaux + (int64_t)it.h * a.m + it.tn * 128 +
+                         half * 64;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) zq[c] = *reinterpret_cast<const uint4*>(zr + c * 8);
+    };
     int it_n = 0;
     for (int item = pair; item < n_items; item += npairs, ++it_n) {
       const WgItem it = wg_item(a, item);
       const uint32_t ab = it_n & 1;
+      const int64_t row = (int64_t)it.tm * 256 + rank * 128 + rloc;
+      // the epilogue's own global inputs do not depend on the MMAs: their loads are issued
+      // before waiting for the accumulator so their latency overlaps the wait
+      uint4 pre[16], pre_z[8];
+      if (EPI == WG_SWIGLU_BWD) {
+#pragma unroll
+        z_load(item, pre_z);
+        for (int c = 0; c < 8; ++c) pre[c] = pre_z[c];
+      }
+      if (EPI == WG_GATE && row < a.M) {
+        const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(a.aux) + row * a.ldaux + it.tn * 256 + half * 128;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pre[c] = *reinterpret_cast<const uint4*>(xr + c * 8);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(bars.accfull + ab, (it_n >> 1) & 1, g))) break;
       tc_fence_after();
-      // this thread's 128 accumulator columns: the SwiGLU products take 64 columns
-      // of H1 (0..127) and the matching 64 of H3 (128..255)
-      uint32_t v[4][32];
       const uint32_t base = tmem + lane_base + ab * 256;
-      if (EPI == WG_SWIGLU_BWD || EPI == WG_SWIGLU_FWD) {
-        tmem_ld32(base + half * 64, v[0]);
-        tmem_ld32(base + half * 64 + 32, v[1]);
-        tmem_ld32(base + 128 + half * 64, v[2]);
-        tmem_ld32(base + 128 + half * 64 + 32, v[3]);
-      } else {
+      const uint32_t accempty_l = ab ? accempty_l1 : accempty_l0;
+      if constexpr (EPI == WG_STORE16 || EPI == WG_STORE_BF16 || EPI == WG_PARTIAL) {
+        // this thread's 128 columns: all TMEM loads, release the buffer, then store
+        uint32_t v[4][32];
 #pragma unroll
         for (int p = 0; p < 4; ++p) tmem_ld32(base + half * 128 + p * 32, v[p]);
-      }
 #pragma unroll
-      for (int p = 0; p < 4; ++p) tmem_ld_wait(v[p]);
-      tc_fence_before();
-      warp_arrive_cluster(ab ? accempty_l1 : accempty_l0);
-
-      const int64_t row = (int64_t)it.tm * 256 + rank * 128 + rloc;
-      if (row >= a.M) continue;
-      if constexpr (EPI == WG_STORE16 || EPI == WG_STORE_BF16) {
-        const int64_t col = (int64_t)it.h * a.out_head + it.tn * 256 + half * 128;
+        for (int p = 0; p < 4; ++p) tmem_ld_wait(v[p]);
+        tc_fence_before();
+        warp_arrive_cluster(accempty_l);
+        if (row >= a.M) continue;
+        if constexpr (EPI == WG_PARTIAL) {
+          // partial[s][mat][h][M][N] (g1, g3: [m][d]; g2: [d][m]), scaled by 1/s
+          const int Nn = it.mat == 2 ? a.m : a.d;
+          const int64_t n = (int64_t)a.m * a.d;
+          float* dst = static_cast<float*>(a.out) + ((int64_t)it.s * 3 + it.mat) * a.heads * n + (int64_t)it.h * n +
+                       row * Nn + it.tn * 256 + half * 128;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+          for (int p = 0; p < 4; ++p)
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint4 x;
-            if (EPI == WG_STORE16) {
-              x = make_uint4(pack_f16x2(__uint_as_float(v[p][c]), __uint_as_float(v[p][c + 1])),
-                             pack_f16x2(__uint_as_float(v[p][c + 2]), __uint_as_float(v[p][c + 3])),
-                             pack_f16x2(__uint_as_float(v[p][c + 4]), __uint_as_float(v[p][c + 5])),
-                             pack_f16x2(__uint_as_float(v[p][c + 6]), __uint_as_float(v[p][c + 7])));
-              *reinterpret_cast<uint4*>(static_cast<__half*>(a.out) + row * a.ldo + col + p * 32 + c) = x;
-            } else {
-              x = make_uint4(pack_bf16x2(__uint_as_float(v[p][c]), __uint_as_float(v[p][c + 1])),
-                             pack_bf16x2(__uint_as_float(v[p][c + 2]), __uint_as_float(v[p][c + 3])),
-                             pack_bf16x2(__uint_as_float(v[p][c + 4]), __uint_as_float(v[p][c + 5])),
-                             pack_bf16x2(__uint_as_float(v[p][c + 6]), __uint_as_float(v[p][c + 7])));
-              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * a.ldo + col + p * 32 + c) = x;
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(dst + p * 32 + c) =
+                  make_float4(__uint_as_float(v[p][c]) * scale, __uint_as_float(v[p][c + 1]) * scale,
+                              __uint_as_float(v[p][c + 2]) * scale, __uint_as_float(v[p][c + 3]) * scale);
+        } else {
+          const int64_t col = (int64_t)it.h * a.out_head + it.tn * 256 + half * 128;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                w4[i] = EPI == WG_STORE16
+                            ? pack_f16x2(__uint_as_float(v[p][c + 2 * i]), __uint_as_float(v[p][c + 2 * i + 1]))
+                            : pack_bf16x2(__uint_as_float(v[p][c + 2 * i]), __uint_as_float(v[p][c + 2 * i + 1]));
+              uint8_t* dst = static_cast<uint8_t*>(a.out) + (row * a.ldo + col + p * 32 + c) * 2;
+              *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
           }
         }
-      } else if constexpr (EPI == WG_PARTIAL) {
-        // partial[s][mat][h][M][N] (g1, g3: [m][d]; g2: [d][m]), scaled by 1/s
-        const int Nn = it.mat == 2 ? a.m : a.d;
-        const int64_t n = (int64_t)a.m * a.d;
-        float* dst = static_cast<float*>(a.out) + ((int64_t)it.s * 3 + it.mat) * a.heads * n + (int64_t)it.h * n +
-                     row * Nn + it.tn * 256 + half * 128;
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-#pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(dst + p * 32 + c) =
-                make_float4(__uint_as_float(v[p][c]) * scale, __uint_as_float(v[p][c + 1]) * scale,
-                            __uint_as_float(v[p][c + 2]) * scale, __uint_as_float(v[p][c + 3]) * scale);
-      } else if constexpr (EPI == WG_SWIGLU_BWD) {
-        // m columns [tn*128 + half*64, +64) of head h
+      } else if constexpr (EPI == WG_SWIGLU_BWD || EPI == WG_SWIGLU_FWD) {
+        // m columns [tn*128 + half*64, +64) of head h, in two 32-column phases: H1 from
+        // accumulator columns half*64 + .., H3 from 128 + half*64 + ..
         const int64_t col = (int64_t)it.h * a.m + it.tn * 128 + half * 64;
-        const __half* zr = static_cast<const __half*>(a.aux) + row * a.ldaux + col;
-        __half* o1 = static_cast<__half*>(a.out) + row * a.ldo + col;
-        __half* o3 = static_cast<__half*>(a.out2) + row * a.ldo + col;
-        __half* ou = static_cast<__half*>(a.out3) + row * a.ldo + col;
+        const float r = (EPI == WG_SWIGLU_FWD && a.rvec && row < a.M) ? a.rvec[row * a.heads + it.h] : 1.f;
 #pragma unroll
-        for (int c8 = 0; c8 < 64; c8 += 8) {
-          float z[8];
-          ld8_f16(zr + c8, z);
-          uint32_t p1[4], p3[4], pu[4];
-#pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            const int cc = c8 + j;
-            const float2 h1 = make_float2(__uint_as_float(v[cc >> 5][cc & 31]), __uint_as_float(v[cc >> 5][(cc & 31) + 1]));
-            const float2 h3 =
-                make_float2(__uint_as_float(v[2 + (cc >> 5)][cc & 31]), __uint_as_float(v[2 + (cc >> 5)][(cc & 31) + 1]));
-            float2 d1, d3, u;
-            swiglu_bwd2(h1, h3, make_float2(z[j], z[j + 1]), d1, d3, u);
-            p1[j >> 1] = pack_f16x2(d1.x, d1.y);
-            p3[j >> 1] = pack_f16x2(d3.x, d3.y);
-            pu[j >> 1] = pack_f16x2(u.x, u.y);
+        for (int ph = 0; ph < 2; ++ph) {
+          uint32_t v1[32], v3[32];
+          tmem_ld32(base + half * 64 + ph * 32, v1);
+          tmem_ld32(base + 128 + half * 64 + ph * 32, v3);
+          tmem_ld_wait(v1);
+          tmem_ld_wait(v3);
+          if (ph == 1) {
+            tc_fence_before();
+            warp_arrive_cluster(accempty_l);
           }
-          *reinterpret_cast<uint4*>(o1 + c8) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
-          *reinterpret_cast<uint4*>(o3 + c8) = make_uint4(p3[0], p3[1], p3[2], p3[3]);
-          *reinterpret_cast<uint4*>(ou + c8) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
-        }
-      } else if constexpr (EPI == WG_SWIGLU_FWD) {
-        const int64_t col = (int64_t)it.h * a.m + it.tn * 128 + half * 64;
-        const float r = a.rvec ? a.rvec[row * a.heads + it.h] : 1.f;
-        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(a.out) + row * a.ldo + col;
+          if (row >= a.M) continue;
 #pragma unroll
-        for (int c8 = 0; c8 < 64; c8 += 8) {
-          uint32_t pk[4];
+          for (int c8 = 0; c8 < 32; c8 += 8) {
+            uint32_t p1[4], p3[4], pu[4];
+            if constexpr (EPI == WG_SWIGLU_BWD) {
+              const uint4 zq = pre[(ph * 32 + c8) >> 3];
+              const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
 #pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            const int cc = c8 + j;
-            const float h1a = r * __uint_as_float(v[cc >> 5][cc & 31]);
-            const float h1b = r * __uint_as_float(v[cc >> 5][(cc & 31) + 1]);
-            const float h3a = r * __uint_as_float(v[2 + (cc >> 5)][cc & 31]);
-            const float h3b = r * __uint_as_float(v[2 + (cc >> 5)][(cc & 31) + 1]);
-            pk[j >> 1] = pack_bf16x2(silu_f(h1a) * h3a, silu_f(h1b) * h3b);
+              for (int j = 0; j < 8; j += 2) {
+                const float2 h1 = make_float2(__uint_as_float(v1[c8 + j]), __uint_as_float(v1[c8 + j + 1]));
+                const float2 h3 = make_float2(__uint_as_float(v3[c8 + j]), __uint_as_float(v3[c8 + j + 1]));
+                float2 d1, d3, u;
+                swiglu_bwd2(h1, h3, unpack_f16x2(zw[j >> 1]), d1, d3, u);
+                p1[j >> 1] = pack_f16x2(d1.x, d1.y);
+                p3[j >> 1] = pack_f16x2(d3.x, d3.y);
+                pu[j >> 1] = pack_f16x2(u.x, u.y);
+              }
+              const int64_t o = row * a.ldo + col + ph * 32 + c8;
+              *reinterpret_cast<uint4*>(static_cast<__half*>(a.out) + o) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+              *reinterpret_cast<uint4*>(static_cast<__half*>(a.out2) + o) = make_uint4(p3[0], p3[1], p3[2], p3[3]);
+              *reinterpret_cast<uint4*>(static_cast<__half*>(a.out3) + o) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; j += 2) {
+                const float h1a = r * __uint_as_float(v1[c8 + j]), h1b = r * __uint_as_float(v1[c8 + j + 1]);
+                const float h3a = r * __uint_as_float(v3[c8 + j]), h3b = r * __uint_as_float(v3[c8 + j + 1]);
+                p1[j >> 1] = pack_bf16x2(silu_f(h1a) * h3a, silu_f(h1b) * h3b);
+              }
+              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * a.ldo + col + ph * 32 + c8) =
+                  make_uint4(p1[0], p1[1], p1[2], p1[3]);
+              (void)p3;
+              (void)pu;
+            }
           }
-          *reinterpret_cast<uint4*>(op + c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       } else if constexpr (EPI == WG_GATE) {
+        // columns [tn*256 + half*128, +128) in four 32-column phases
         const int64_t col = (int64_t)it.tn * 256 + half * 128;
-        const float ri = a.rvec[row];
-        const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(a.aux) + row * a.ldaux + col;
-        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(a.out) + row * a.ldo + col;
+        const float ri = row < a.M ? a.rvec[row] : 0.f;
 #pragma unroll
-        for (int c8 = 0; c8 < 128; c8 += 8) {
-          float x[8];
-          ld8_bf16(xr + c8, x);
-          uint32_t pk[4];
-#pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            const int cc = c8 + j;
-            const float ga = __uint_as_float(v[cc >> 5][cc & 31]), gb = __uint_as_float(v[cc >> 5][(cc & 31) + 1]);
-            pk[j >> 1] = pack_bf16x2(x[j] * ri * silu_f(ga), x[j + 1] * ri * silu_f(gb));
+        for (int ph = 0; ph < 4; ++ph) {
+          uint32_t v[32];
+          tmem_ld32(base + half * 128 + ph * 32, v);
+          tmem_ld_wait(v);
+          if (ph == 3) {
+            tc_fence_before();
+            warp_arrive_cluster(accempty_l);
           }
-          *reinterpret_cast<uint4*>(op + c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          if (row >= a.M) continue;
+#pragma unroll
+          for (int c8 = 0; c8 < 32; c8 += 8) {
+            const uint4 q = pre[(ph * 32 + c8) >> 3];
+            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float xa = __uint_as_float(w4[i] << 16), xb = __uint_as_float(w4[i] & 0xffff0000u);
+              const float ga = __uint_as_float(v[c8 + 2 * i]), gb = __uint_as_float(v[c8 + 2 * i + 1]);
+              pk[i] = pack_bf16x2(xa * ri * silu_f(ga), xb * ri * silu_f(gb));
+            }
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * a.ldo + col + ph * 32 + c8) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      } else if constexpr (EPI == WG_NSOUT) {
+        // C = alpha acc + beta Cin for matrix h (rows M, stride ldo), plus C's bf16 hi and lo
+        // parts (the next product's split operands), four 32-column phases
+        const int64_t mbase = (int64_t)it.h * a.M * a.ldo + row * a.ldo + it.tn * 256 + half * 128;
+        const float* cin = static_cast<const float*>(a.aux);
+#pragma unroll
+        for (int ph = 0; ph < 4; ++ph) {
+          float4 ci[8];
+          if (cin) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) ci[q] = *reinterpret_cast<const float4*>(cin + mbase + ph * 32 + q * 4);
+          }
+          uint32_t v[32];
+          tmem_ld32(base + half * 128 + ph * 32, v);
+          tmem_ld_wait(v);
+          if (ph == 3) {
+            tc_fence_before();
+            warp_arrive_cluster(accempty_l);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 c = cin ? ci[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+            float o[4];
+            o[0] = fmaf(a.alpha, __uint_as_float(v[4 * q + 0]), a.beta * c.x);
+            o[1] = fmaf(a.alpha, __uint_as_float(v[4 * q + 1]), a.beta * c.y);
+            o[2] = fmaf(a.alpha, __uint_as_float(v[4 * q + 2]), a.beta * c.z);
+            o[3] = fmaf(a.alpha, __uint_as_float(v[4 * q + 3]), a.beta * c.w);
+            const int64_t off = mbase + ph * 32 + q * 4;
+            *reinterpret_cast<float4*>(static_cast<float*>(a.out) + off) = make_float4(o[0], o[1], o[2], o[3]);
+            uint32_t hi[2], lo[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              hi[e] = pack_bf16x2(o[2 * e], o[2 * e + 1]);
+              const float h0 = __uint_as_float(hi[e] << 16), h1 = __uint_as_float(hi[e] & 0xffff0000u);
+              lo[e] = pack_bf16x2(o[2 * e] - h0, o[2 * e + 1] - h1);
+            }
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out2) + off) = make_uint2(hi[0], hi[1]);
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out3) + off) = make_uint2(lo[0], lo[1]);
+          }
         }
       }
     }
@@ -474,6 +558,20 @@ __global__ void __launch_bounds__(256) k_rms_rows(const __nv_bfloat16* __restric
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) rinv[t] = 1.0f / sqrtf(ss / (float)D + eps);
+  }
+}
+
+// bf16 hi and lo parts of an fp32 array: hi = bf16(x), lo = bf16(x - hi) (n a multiple of 4).
+__global__ void k_split_bf16(const float* __restrict__ x, __nv_bfloat16* __restrict__ hi,
+                             __nv_bfloat16* __restrict__ lo, int64_t n) {
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; i < n;
+       i += (int64_t)gridDim.x * blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    const uint32_t h0 = pack_bf16x2(v.x, v.y), h1 = pack_bf16x2(v.z, v.w);
+    const uint32_t l0 = pack_bf16x2(v.x - __uint_as_float(h0 << 16), v.y - __uint_as_float(h0 & 0xffff0000u));
+    const uint32_t l1 = pack_bf16x2(v.z - __uint_as_float(h1 << 16), v.w - __uint_as_float(h1 & 0xffff0000u));
+    *reinterpret_cast<uint2*>(hi + i) = make_uint2(h0, h1);
+    *reinterpret_cast<uint2*>(lo + i) = make_uint2(l0, l1);
   }
 }
 

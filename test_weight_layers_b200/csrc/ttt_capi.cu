@@ -98,6 +98,8 @@ struct Ws {
   __half* dh1;         // dL/dh1 (the apply's P, bf16, reuses this buffer)
   __half* dh3;         // dL/dh3
   __half* u16;         // u
+  // wide-head Newton-Schulz: bf16 hi/lo parts of X (ping-pong), A and B = c A A + b A
+  __nv_bfloat16 *xh, *xl, *x2h, *x2l, *ah, *al, *bh, *bl;
   size_t total;
   int s_max;
 };
@@ -162,6 +164,11 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_dh1 = wide ? take(tokm) : 0;
   const size_t o_dh3 = wide ? take(tokm) : 0;
   const size_t o_u = wide ? take(tokm) : 0;
+  const size_t nsx = wide ? 3 * n * 2 : 0, nsa = wide ? 3 * H * r * r * 2 : 0;
+  const size_t o_xh = wide ? take(nsx) : 0, o_xl = wide ? take(nsx) : 0;
+  const size_t o_x2h = wide ? take(nsx) : 0, o_x2l = wide ? take(nsx) : 0;
+  const size_t o_ah = wide ? take(nsa) : 0, o_al = wide ? take(nsa) : 0;
+  const size_t o_bh = wide ? take(nsa) : 0, o_bl = wide ? take(nsa) : 0;
   w.total = off;
   uint8_t* b = static_cast<uint8_t*>(base);
   if (b) {
@@ -191,6 +198,15 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
         w.dh1 = reinterpret_cast<__half*>(b + o_dh1);
         w.dh3 = reinterpret_cast<__half*>(b + o_dh3);
         w.u16 = reinterpret_cast<__half*>(b + o_u);
+        auto bf = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(b + o); };
+        w.xh = bf(o_xh);
+        w.xl = bf(o_xl);
+        w.x2h = bf(o_x2h);
+        w.x2l = bf(o_x2l);
+        w.ah = bf(o_ah);
+        w.al = bf(o_al);
+        w.bh = bf(o_bh);
+        w.bl = bf(o_bl);
       }
     }
   }
@@ -526,8 +542,81 @@ bool tmap_k(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, uin
                    f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 // MN-major operand map over token rows: 64 x 64 boxes (64 columns of 64 tokens).
-bool tmap_mn(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows) {
-  return tmap_bf16(tm, base, cols, rows, cols * 2, 64, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+bool tmap_mn(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, bool f16 = true) {
+  return tmap_bf16(tm, base, cols, rows, cols * 2, 64, 64,
+                   f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+// Newton-Schulz iterations of the wide-head path on the 2-SM GEMM kernel: nb matrices
+// X (r x c, fp32, stacked) -> X after `iters` steps.  Every product takes split bf16
+// operands (hi + lo) as three K segments, hi.hi + hi.lo + lo.hi, and its epilogue
+// writes the fp32 result with its own hi/lo parts for the next product.
+int run_ns_iters_wide(const ttt_ns_cfg& ns, int r, int c, int nb, const Ws& w, float*& X, float*& X2,
+                      cudaStream_t s) {
+  const int64_t nx = (int64_t)nb * r * c;
+  __nv_bfloat16 *xh = w.xh, *xl = w.xl, *x2h = w.x2h, *x2l = w.x2l;
+  k_split_bf16<<<grid1d(nx / 4, 256), 256, 0, s>>>(X, xh, xl, nx);
+  TTT_LAUNCHED();
+  CUtensorMap tAh, tAl, tBh, tBl;
+  const uint64_t R = (uint64_t)nb * r;
+  if (!tmap_k(&tAh, w.ah, (uint64_t)r, R, (uint64_t)r, false) || !tmap_k(&tAl, w.al, (uint64_t)r, R, (uint64_t)r, false) ||
+      !tmap_k(&tBh, w.bh, (uint64_t)r, R, (uint64_t)r, false) || !tmap_k(&tBl, w.bl, (uint64_t)r, R, (uint64_t)r, false))
+    return TTT_ERR_CUDA;
+  for (int it = 0; it < ns.iters; ++it) {
+    CUtensorMap tXh, tXl, tXmh, tXml;
+    if (!tmap_k(&tXh, xh, (uint64_t)c, R, (uint64_t)c, false) || !tmap_k(&tXl, xl, (uint64_t)c, R, (uint64_t)c, false) ||
+        !tmap_mn(&tXmh, xh, (uint64_t)c, R, false) || !tmap_mn(&tXml, xl, (uint64_t)c, R, false))
+      return TTT_ERR_CUDA;
+    WgArgs g = wg_args();
+    g.M = r;
+    g.heads = nb;
+    g.a_row_head = r;
+    g.idesc = idesc_bf16(256, 256, false, false);
+    // A = X X^T (B rows = X rows)
+    WgArgs a1 = g;
+    a1.mt = a1.nt = r / 256;
+    a1.kblocks = 3 * (c / 64);
+    a1.b_head = r;
+    a1.out = w.A;
+    a1.out2 = w.ah;
+    a1.out3 = w.al;
+    a1.ldo = r;
+    a1.alpha = 1.f;
+    a1.beta = 0.f;
+    TTT_TRY((launch_wgemm<WG_NSOUT, false, false>(tXh, tXl, tXl, tXh, tXl, a1, a1.mt * a1.nt * nb, w, s)));
+    // B = c A A + b A (A symmetric: its rows serve as the B operand's rows)
+    WgArgs a2 = g;
+    a2.mt = a2.nt = r / 256;
+    a2.kblocks = 3 * (r / 64);
+    a2.b_head = r;
+    a2.out = w.B;
+    a2.out2 = w.bh;
+    a2.out3 = w.bl;
+    a2.ldo = r;
+    a2.aux = w.A;
+    a2.alpha = ns.c;
+    a2.beta = ns.b;
+    TTT_TRY((launch_wgemm<WG_NSOUT, false, false>(tAh, tAl, tAl, tAh, tAl, a2, a2.mt * a2.nt * nb, w, s)));
+    // X' = B X + a X (X rows are the K rows of the MN-major B operand)
+    WgArgs a3 = g;
+    a3.mt = r / 256;
+    a3.nt = c / 256;
+    a3.kblocks = 3 * (r / 64);
+    a3.b_y_head = r;
+    a3.out = X2;
+    a3.out2 = x2h;
+    a3.out3 = x2l;
+    a3.ldo = c;
+    a3.aux = X;
+    a3.alpha = 1.f;
+    a3.beta = ns.a;
+    a3.idesc = idesc_bf16(256, 256, false, true);
+    TTT_TRY((launch_wgemm<WG_NSOUT, false, true>(tBh, tBl, tBl, tXmh, tXml, a3, a3.mt * a3.nt * nb, w, s)));
+    std::swap(X, X2);
+    std::swap(xh, x2h);
+    std::swap(xl, x2l);
+  }
+  return TTT_OK;
 }
 
 // Gradient of the wide path from the prepared fp16 operands K^, V' ([T][H*d]):
@@ -861,6 +950,8 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
         bool unused = false;
         TTT_TRY(r == 192 ? ns_cluster_launch<192>(c, nb, ns, w, s, false, &unused)
                          : ns_cluster_launch<128>(c, nb, ns, w, s, false, &unused));
+      } else if (wide_dims(d)) {
+        TTT_TRY(run_ns_iters_wide(ns, r, c, nb, w, X, X2, s));
       } else {
         TTT_TRY(run_ns_iters_tc(ns, r, c, nb, w, X, X2, s));
       }

@@ -171,6 +171,30 @@ def test_step_matches_oracle(dt, d, m, iters, renorm, lr):
     del dtype
 
 
+# the wide-head path's Newton-Schulz: products on 2-SM tensor-core pairs from split
+# bf16 operands (three K segments), for r x c = 256 x 512 (tall and wide gradients)
+# and ZipMap's 1,024 x 2,048
+@pytest.mark.parametrize("H,d,m,iters,renorm,lr", [(2, 256, 512, 5, 1, 1.0), (1, 512, 256, 3, 0, 0.5),
+                                                   (1, 1024, 2048, 5, 1, 1.0)])
+def test_step_matches_oracle_wide(H, d, m, iters, renorm, lr):
+    W = DevWeights(*rand_weights(H, d, m, 44))
+    Wo = W.oracle()
+    K = rand_tokens(300, H, d, torch.float32, 45)
+    V = rand_tokens(300, H, d, torch.float32, 46)
+    G = O.grad(Wo, O.l2norm_heads(f64(K), H, d), f64(V), f64(rand_eta(300, H, 47, 1.0)))
+    Gflat = torch.from_numpy(np.concatenate([G.W1.ravel(), G.W3.ravel(), G.W2.ravel()])).float()
+    dm = T.dims(H, d, m)
+    ws = T.workspace(dm, 0, T.TTT_BF16)
+    cfg = O.NSConfig(iters=iters, renorm=renorm, lr=lr)
+    T.ttt_step(W.abi, Gflat.cuda(), T.ns_cfg(iters=iters, renorm=renorm, lr=lr), dm, T.TTT_BF16, ws)
+    check_status(ws)
+    n = H * m * d
+    ref = O.muon_step(Wo, O.FastWeights(f64(Gflat[:n].reshape(H, m, d)), f64(Gflat[n:2 * n].reshape(H, m, d)),
+                                        f64(Gflat[2 * n:].reshape(H, d, m))), cfg)
+    errs = weight_errors(W.oracle(), ref)
+    assert max(errs) < 1e-4, errs
+
+
 def test_update_eta_zero_keeps_weights_bf16():
     H, d, m, T_ = 2, 192, 128, 500
     W = DevWeights(*rand_weights(H, d, m, 50))
