@@ -331,6 +331,11 @@ def run_ours(args, cfg):
         for w, w0 in zip(W, W0):
             w.copy_(w0, non_blocking=True)
         Vuse = Vx
+        if cfg.conv and world == 1 and not cfg.chunk and dcode == T.TTT_BF16:
+            # ShortConv2D folded into the update's operand preparation
+            T.ttt_update_conv(Wabi, Kx, Vx, ex, Tn, cfg.steps, ns, taps, cfg.grid_h, cfg.grid_w, dm, io, ws)
+            T.ttt_apply(Wabi, Qx, Ox, Ta, dm, io, ws)
+            return
         if cfg.conv:
             T.ttt_shortconv2d(Vx, Vc, taps, cfg.frames, cfg.grid_h, cfg.grid_w, D)
             Vuse = Vc
@@ -345,6 +350,8 @@ def run_ours(args, cfg):
             sharded_layer(
                 Tn, cfg.steps,
                 grad=lambda t0, t1: (T.ttt_grad(Wabi, Kx[t0:t1], Vuse[t0:t1], ex[t0:t1], t1 - t0, dm, io, G, ws), G)[1],
+                grad_again=lambda t0, t1: (T.ttt_grad_prepared(Wabi, Kx[t0:t1], Vuse[t0:t1], ex[t0:t1], t1 - t0, dm,
+                                                               io, G, ws), G)[1],
                 allreduce=lambda g_: dist.all_reduce(g_),
                 step=lambda g_: T.ttt_step(Wabi, g_, ns, dm, dcode, ws),
                 apply=(lambda t0, t1: T.ttt_apply(Wabi, Qx[t0:t1], Ox[t0:t1], t1 - t0, dm, io, ws))

@@ -141,6 +141,17 @@ int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int6
              ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, float* G,
              void* ws, size_t ws_bytes, void* stream);
 
+/* ttt_grad without the operand preparation: the workspace must hold what the last
+ * ttt_grad (or ttt_grad_prepared) on it prepared, for the same K, V, eta, T and io
+ * (bf16 mode: the fp16 K^ and V' and the |eta| maxima; fp32 mode: the per-token key
+ * norms), while W may have changed since (e.g. by ttt_step).  This is the second
+ * inner step of a multi-device update (ttt_grad, sum of G across devices, ttt_step,
+ * then this): it saves the preparation pass, a read of K and V and a write of their
+ * fp16 copies.  The fp16 weight copy is refreshed from W as in ttt_grad. */
+int ttt_grad_prepared(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T,
+                      ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype, float* G,
+                      void* ws, size_t ws_bytes, void* stream);
+
 /* Muon step from a given gradient G (layout as in ttt_grad); updates W in place.
  * Newton-Schulz precision: TTT_FP32 multiplies in fp32 on the CUDA cores;
  * TTT_BF16 multiplies on the tensor cores from split operands (each fp32
@@ -154,6 +165,18 @@ int ttt_step(ttt_weights W, const float* G, const ttt_ns_cfg* ns, ttt_dims dims,
 int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, int steps,
                const ttt_ns_cfg* ns, ttt_dims dims, const ttt_io_cfg* io, ttt_dtype dtype,
                void* ws, size_t ws_bytes, void* stream);
+
+/* TTTUpdate with ShortConv2D on V (VGG-T3 key design 2) folded into the update's
+ * operand preparation: the same result as ttt_shortconv2d(V -> V', taps, T /
+ * (grid_h * grid_w) frames of grid_h x grid_w, act) followed by ttt_update(K, V'),
+ * except that the convolved values are rounded once, to the update's fp16 value
+ * operand, instead of first to bf16 -- V' itself is never written.  taps: device
+ * float [H*d][3][3].  TTT_BF16 only; T must be whole frames; the head dim d must be
+ * a multiple of 64 and a frame row must fit a shared-memory band (true for grids up
+ * to several hundred tokens wide), else TTT_ERR_UNSUPPORTED. */
+int ttt_update_conv(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, int steps,
+                    const ttt_ns_cfg* ns, const float* taps, int grid_h, int grid_w, int act, ttt_dims dims,
+                    const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
 /* Apply: O[i] = f_W(q_i) for T query rows (Q and O may not alias). */
 int ttt_apply(ttt_weights W, const void* Q, void* O, int64_t T, ttt_dims dims,

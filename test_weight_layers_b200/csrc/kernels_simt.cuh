@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
         hv[k] = v < nvt ? v * VN / d : -1;
         if (hv[k] >= 0) {
           xk[k] = __ldg(reinterpret_cast<const uint4*>(krow + v * VN));
-          xv[k] = __ldg(reinterpret_cast<const uint4*>(vrow + v * VN));
+          xv[k] = Vh ? __ldg(reinterpret_cast<const uint4*>(vrow + v * VN)) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
       float inv[RN_MAX_VEC];
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
             pv[i] = pack_f16x2(fv.x * vek, fv.y * vek);
           }
           *reinterpret_cast<uint4*>(Kh + t * HD + (lane + 32 * k) * VN) = ok;
-          *reinterpret_cast<uint4*>(Vh + t * HD + (lane + 32 * k) * VN) = ov;
+          if (Vh) *reinterpret_cast<uint4*>(Vh + t * HD + (lane + 32 * k) * VN) = ov;
         }
       }
     } else {
@@ -301,14 +301,14 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
         for (int v = lane; v < d / VN; v += 32) {
           float x[VN], y[VN];
           load16(krow + h * d + v * VN, x);
-          load16(vrow + h * d + v * VN, y);
+          if (Vh) load16(vrow + h * d + v * VN, y);
 #pragma unroll
           for (int i = 0; i < VN; ++i) {
             x[i] *= r;
-            y[i] *= ve;
+            y[i] = Vh ? y[i] * ve : 0.f;
           }
           store16_h(Kh + t * HD + h * d + v * VN, x);
-          store16_h(Vh + t * HD + h * d + v * VN, y);
+          if (Vh) store16_h(Vh + t * HD + h * d + v * VN, y);
         }
       }
     }
@@ -513,10 +513,15 @@ __device__ __forceinline__ void bf16x8_f2(const uint4 q, float2 (&f)[4]) {
   for (int e = 0; e < 4; ++e) f[e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
 }
 
+// FUSE = false: the ShortConv2D output V' in bf16 (ttt_shortconv2d).  FUSE = true: the
+// update's fp16 value operand -s eta_(t,h) V' directly (dense [T][C], head h = c / d), so
+// V' never makes a bf16 round trip through HBM; s is the value scale of eta_part.
+template <bool FUSE>
 __global__ void __launch_bounds__(256, 2) k_shortconv_band2(const __nv_bfloat16* __restrict__ V, int64_t ldv,
-                                                         __nv_bfloat16* __restrict__ out, int64_t ldo,
+                                                         void* __restrict__ out, int64_t ldo,
                                                          const float* __restrict__ taps, int N, int gh, int gw, int C,
-                                                         int act, int BR) {
+                                                         int act, int BR, const float* __restrict__ eta,
+                                                         const float* __restrict__ eta_part, int H, int d) {
   constexpr int TPT = CONV_GROUP / 8;  // threads (8-channel chunks) per token
   constexpr int NL = 256 / TPT;        // output pairs per pass
   extern __shared__ __align__(16) uint8_t cdyn[];
@@ -533,6 +538,12 @@ __global__ void __launch_bounds__(256, 2) k_shortconv_band2(const __nv_bfloat16*
   const int chunk = tid % TPT, tl = tid / TPT;
   const int c0 = g0 + chunk * 8;
   const int ntok = gh * gw, nbands = (gh + BR - 1) / BR, nstrips = (gw + CONV2_SX - 1) / CONV2_SX;
+  float vscale = 0.f;
+  if (FUSE) {
+    float inv_unused;
+    value_scale(eta_parts_max(eta_part), vscale, inv_unused);
+  }
+  const int head = FUSE ? c0 / d : 0;
   __syncthreads();
   float2 wr[9][4];  // this thread's taps as channel pairs, in registers for all its outputs
 #pragma unroll
@@ -606,12 +617,28 @@ __global__ void __launch_bounds__(256, 2) k_shortconv_band2(const __nv_bfloat16*
               a1[i].y = a1[i].y / (1.0f + expf(-a1[i].y));
             }
           }
-          __nv_bfloat16* o = out + (frame0 + (int64_t)(y0 + ry) * gw + x0) * ldo + c0;
-          *reinterpret_cast<uint4*>(o) = make_uint4(pack_bf16x2(a0[0].x, a0[0].y), pack_bf16x2(a0[1].x, a0[1].y),
-                                                    pack_bf16x2(a0[2].x, a0[2].y), pack_bf16x2(a0[3].x, a0[3].y));
-          if (x0 + 1 < gw)
-            *reinterpret_cast<uint4*>(o + ldo) = make_uint4(pack_bf16x2(a1[0].x, a1[0].y), pack_bf16x2(a1[1].x, a1[1].y),
-                                                            pack_bf16x2(a1[2].x, a1[2].y), pack_bf16x2(a1[3].x, a1[3].y));
+          const int64_t t0 = frame0 + (int64_t)(y0 + ry) * gw + x0;
+          if (FUSE) {
+            const float s0 = -vscale * __ldg(eta + t0 * H + head);
+            __half* o = static_cast<__half*>(out) + t0 * ldo + c0;
+            *reinterpret_cast<uint4*>(o) =
+                make_uint4(pack_f16x2(a0[0].x * s0, a0[0].y * s0), pack_f16x2(a0[1].x * s0, a0[1].y * s0),
+                           pack_f16x2(a0[2].x * s0, a0[2].y * s0), pack_f16x2(a0[3].x * s0, a0[3].y * s0));
+            if (x0 + 1 < gw) {
+              const float s1 = -vscale * __ldg(eta + (t0 + 1) * H + head);
+              *reinterpret_cast<uint4*>(o + ldo) =
+                  make_uint4(pack_f16x2(a1[0].x * s1, a1[0].y * s1), pack_f16x2(a1[1].x * s1, a1[1].y * s1),
+                             pack_f16x2(a1[2].x * s1, a1[2].y * s1), pack_f16x2(a1[3].x * s1, a1[3].y * s1));
+            }
+          } else {
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out) + t0 * ldo + c0;
+            *reinterpret_cast<uint4*>(o) = make_uint4(pack_bf16x2(a0[0].x, a0[0].y), pack_bf16x2(a0[1].x, a0[1].y),
+                                                      pack_bf16x2(a0[2].x, a0[2].y), pack_bf16x2(a0[3].x, a0[3].y));
+            if (x0 + 1 < gw)
+              *reinterpret_cast<uint4*>(o + ldo) =
+                  make_uint4(pack_bf16x2(a1[0].x, a1[0].y), pack_bf16x2(a1[1].x, a1[1].y),
+                             pack_bf16x2(a1[2].x, a1[2].y), pack_bf16x2(a1[3].x, a1[3].y));
+          }
         }
       }
       __syncthreads();  // `cur` may be refilled by the prefetch of band bi + 2

@@ -151,12 +151,20 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_gram = take((size_t)std::max(NS_GRAM_SPLIT, NSM_GRAM_SPLIT_MAX) * 3 * H * r * r * 4);
   const size_t o_norms = take(3 * H * NORM_PARTS * 4);
   const size_t o_stepn = take(3 * H * NORM_PARTS * 2 * 4);
-  const size_t o_rk = take((size_t)std::max<int64_t>(T, 1) * H * 4);
-  const size_t o_rq = take((size_t)std::max<int64_t>(T, 1) * H * 4);
+  // every buffer whose size does not depend on T comes first, so its offset is the same
+  // for any T (ttt_step carves with T = 0 beside ttt_grad's T-token layout)
   const bool tc = dt == TTT_BF16;
+  const bool wide = tc && wide_dims(dm);
   const size_t o_wsh16 = tc ? take(3 * n * 2) : 0;
   const size_t o_etap = tc ? take(ETA_PARTS * 4) : 0;
-  const bool wide = tc && wide_dims(dm);
+  const size_t nsx = wide ? 3 * n * 2 : 0, nsa = wide ? 3 * H * r * r * 2 : 0;
+  const size_t o_xh = wide ? take(nsx) : 0, o_xl = wide ? take(nsx) : 0;
+  const size_t o_x2h = wide ? take(nsx) : 0, o_x2l = wide ? take(nsx) : 0;
+  const size_t o_ah = wide ? take(nsa) : 0, o_al = wide ? take(nsa) : 0;
+  const size_t o_bh = wide ? take(nsa) : 0, o_bl = wide ? take(nsa) : 0;
+  // per-token buffers
+  const size_t o_rk = take((size_t)std::max<int64_t>(T, 1) * H * 4);
+  const size_t o_rq = take((size_t)std::max<int64_t>(T, 1) * H * 4);
   const size_t tokd = (size_t)std::max<int64_t>(T, 1) * H * d * 2, tokm = (size_t)std::max<int64_t>(T, 1) * H * m * 2;
   const size_t o_kh = tc ? take(tokd) : 0;
   const size_t o_vh = tc ? take(tokd) : 0;
@@ -164,11 +172,6 @@ Ws carve(void* base, const ttt_dims& dm, int64_t T, ttt_dtype dt) {
   const size_t o_dh1 = wide ? take(tokm) : 0;
   const size_t o_dh3 = wide ? take(tokm) : 0;
   const size_t o_u = wide ? take(tokm) : 0;
-  const size_t nsx = wide ? 3 * n * 2 : 0, nsa = wide ? 3 * H * r * r * 2 : 0;
-  const size_t o_xh = wide ? take(nsx) : 0, o_xl = wide ? take(nsx) : 0;
-  const size_t o_x2h = wide ? take(nsx) : 0, o_x2l = wide ? take(nsx) : 0;
-  const size_t o_ah = wide ? take(nsa) : 0, o_al = wide ? take(nsa) : 0;
-  const size_t o_bh = wide ? take(nsa) : 0, o_bl = wide ? take(nsa) : 0;
   w.total = off;
   uint8_t* b = static_cast<uint8_t*>(base);
   if (b) {
@@ -349,6 +352,18 @@ int launch_rownorm_any(const void* X, int64_t ld, int64_t rows, const ttt_dims& 
   return launch_rownorm<float>((float*)X, ld, rows, d, r_out, 0, s);
 }
 
+// Rows per band of the two-output bf16 ShortConv2D kernel: the largest band that keeps two
+// CTAs per SM (or one, for very wide frames); 0 when not even a band of one row fits.
+int conv2_band_rows(int gh, int gw) {
+  const size_t fixed = 9 * CONV_GROUP * sizeof(float);
+  const size_t row2 = (size_t)conv2_row_slots(gw) * CONV_GROUP * 2;
+  for (size_t budget : {(size_t)110 * 1024, (size_t)220 * 1024}) {
+    const int64_t br = (int64_t)((budget - fixed) / (2 * row2)) - 2;
+    if (br >= 1) return (int)std::min<int64_t>(br, gh);
+  }
+  return 0;
+}
+
 // ShortConv2D launch: the banded shared-memory kernel with the largest band
 // that keeps two CTAs per SM (or one, for very wide frames); the direct kernel
 // for frames too wide for one band of three rows.
@@ -369,20 +384,12 @@ int launch_conv_any(const void* V, int64_t ldv, void* Vout, int64_t ldo, const f
   ProfScope ps(TTT_PROF_CONV, s);
   if (dt == TTT_BF16) {
     // the two-outputs-per-thread bf16 kernel, same band choice with its padded rows
-    const size_t row2 = (size_t)conv2_row_slots(gw) * CONV_GROUP * 2;
-    int BR2 = 0;
-    for (size_t budget : {(size_t)110 * 1024, (size_t)220 * 1024}) {
-      const int64_t br = (int64_t)((budget - fixed) / (2 * row2)) - 2;
-      if (br >= 1) {
-        BR2 = (int)std::min<int64_t>(br, gh);
-        break;
-      }
-    }
+    const int BR2 = conv2_band_rows(gh, gw);
     if (BR2 >= 1) {
       const size_t smem = conv2_band_smem(BR2, gw);
-      TTT_CHECK(cudaFuncSetAttribute(k_shortconv_band2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-      k_shortconv_band2<<<grid, 256, smem, s>>>((const __nv_bfloat16*)V, ldv, (__nv_bfloat16*)Vout, ldo, taps, (int)N,
-                                                gh, gw, C, act, BR2);
+      TTT_CHECK(cudaFuncSetAttribute(k_shortconv_band2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      k_shortconv_band2<false><<<grid, 256, smem, s>>>((const __nv_bfloat16*)V, ldv, Vout, ldo, taps, (int)N, gh, gw, C,
+                                                       act, BR2, nullptr, nullptr, 1, 1);
       TTT_LAUNCHED();
       return TTT_OK;
     }
@@ -479,6 +486,27 @@ struct UpdOperands {
   int64_t ldv;
   const float* rk;
 };
+
+// The fp16 gradient operands of N frames with ShortConv2D on V fused into the value
+// operand: K^ from the preparation kernel (K only), V' = -s eta conv(V) straight from the
+// conv kernel (bf16 mode; the |eta| maxima must be in w.etapart).  Returns
+// TTT_ERR_UNSUPPORTED when the frames are too wide for a row band.
+int launch_conv_prep(const void* K, int64_t ldk, const void* V, int64_t ldv, const float* taps, int64_t N, int gh,
+                     int gw, int act, const float* eta, int l2norm, const ttt_dims& d, const Ws& w, cudaStream_t s) {
+  const int C = d.heads * d.d;
+  const int BR2 = conv2_band_rows(gh, gw);
+  if (BR2 < 1 || d.d % CONV_GROUP) return TTT_ERR_UNSUPPORTED;
+  const int64_t T = N * gh * gw;
+  TTT_TRY(launch_prep_kv(K, ldk, nullptr, 0, eta, T, d, l2norm, w, w.kh16, nullptr, s));
+  const size_t smem = conv2_band_smem(BR2, gw);
+  const dim3 grid((C + CONV_GROUP - 1) / CONV_GROUP, (unsigned)std::min<int64_t>(N, 65535));
+  ProfScope ps(TTT_PROF_CONV, s);
+  TTT_CHECK(cudaFuncSetAttribute(k_shortconv_band2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  k_shortconv_band2<true><<<grid, 256, smem, s>>>((const __nv_bfloat16*)V, ldv, w.vh16, C, taps, (int)N, gh, gw, C, act,
+                                                  BR2, eta, w.etapart, d.heads, d.d);
+  TTT_LAUNCHED();
+  return TTT_OK;
+}
 
 // Operands of the gradient kernels for T tokens: fp16 K^/V' copies in bf16 mode
 // (V' carries the per-token weights eta and the value scale s; w.etapart the
@@ -1199,6 +1227,30 @@ int ttt_grad(ttt_weights W, const void* K, const void* V, const float* eta, int6
   return run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, io->qk_l2norm, T, dims, dtype, w, G, s);
 }
 
+int ttt_grad_prepared(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, ttt_dims dims,
+                      const ttt_io_cfg* io, ttt_dtype dtype, float* G, void* ws, size_t ws_bytes, void* stream) {
+  TTT_TRY(check_common(dims, dtype, T, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  if (!io) io = &kDefaultIo;
+  const int64_t ldk = eff_ld(io->ld_k, dims), ldv = eff_ld(io->ld_v, dims);
+  TTT_TRY(check_tokens(K, ldk, dims, dtype, T));
+  TTT_TRY(check_tokens(V, ldv, dims, dtype, T));
+  if (!G) return TTT_ERR_INVALID;
+  if (!aligned16(G)) return TTT_ERR_ALIGN;
+  if (T > 0 && !eta) return TTT_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  Ws w = carve(ws, dims, T, dtype);
+  UpdOperands op;
+  if (dtype == TTT_BF16) {
+    const int64_t hd = (int64_t)dims.heads * dims.d;
+    op = {w.kh16, hd, w.vh16, hd, nullptr};
+    TTT_TRY(launch_shadow(W, w, dims, s));
+  } else {
+    op = {K, ldk, V, ldv, io->qk_l2norm && T > 0 ? w.rk : nullptr};
+  }
+  return run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, io->qk_l2norm, T, dims, dtype, w, G, s);
+}
+
 int ttt_step(ttt_weights W, const float* G, const ttt_ns_cfg* ns, ttt_dims dims, ttt_dtype dtype, void* ws,
              size_t ws_bytes, void* stream) {
   TTT_TRY(check_common(dims, dtype, 0, ws, ws_bytes));
@@ -1229,6 +1281,36 @@ int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, in
   if (dtype == TTT_BF16) TTT_TRY(launch_shadow(W, w, dims, s));
   for (int st = 0; st < steps; ++st) {
     TTT_TRY(run_grad(W, op.K, op.ldk, op.V, op.ldv, eta, op.rk, io->qk_l2norm, T, dims, dtype, w, w.G, s));
+    TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
+  }
+  return TTT_OK;
+}
+
+int ttt_update_conv(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, int steps,
+                    const ttt_ns_cfg* ns, const float* taps, int grid_h, int grid_w, int act, ttt_dims dims,
+                    const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream) {
+  TTT_TRY(check_common(dims, dtype, T, ws, ws_bytes));
+  TTT_TRY(check_weights(W));
+  TTT_TRY(check_ns(ns));
+  if (steps < 0 || grid_h < 1 || grid_w < 1 || (act != 0 && act != 1)) return TTT_ERR_INVALID;
+  if (T % ((int64_t)grid_h * grid_w)) return TTT_ERR_INVALID;
+  if (dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
+  if (!io) io = &kDefaultIo;
+  const int64_t ldk = eff_ld(io->ld_k, dims), ldv = eff_ld(io->ld_v, dims);
+  TTT_TRY(check_tokens(K, ldk, dims, dtype, T));
+  TTT_TRY(check_tokens(V, ldv, dims, dtype, T));
+  if (T > 0 && (!eta || !taps)) return TTT_ERR_INVALID;
+  if (T == 0 || steps == 0) return TTT_OK;
+  if (conv2_band_rows(grid_h, grid_w) < 1 || dims.d % CONV_GROUP) return TTT_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  Ws w = carve(ws, dims, T, dtype);
+  TTT_TRY(launch_eta_absmax(eta, T, dims, w, s));
+  TTT_TRY(launch_conv_prep(K, ldk, V, ldv, taps, T / ((int64_t)grid_h * grid_w), grid_h, grid_w, act, eta,
+                           io->qk_l2norm, dims, w, s));
+  TTT_TRY(launch_shadow(W, w, dims, s));
+  const int64_t hd = (int64_t)dims.heads * dims.d;
+  for (int st = 0; st < steps; ++st) {
+    TTT_TRY(run_grad(W, w.kh16, hd, w.vh16, hd, eta, nullptr, io->qk_l2norm, T, dims, dtype, w, w.G, s));
     TTT_TRY(run_step(W, w.G, *ns, dims, dtype, w, s));
   }
   return TTT_OK;

@@ -18,7 +18,8 @@ from typing import Callable, Optional
 
 def sharded_layer(n_tokens: int, steps: int, grad: Callable[[int, int], object],
                   allreduce: Callable[[object], None], step: Callable[[object], None],
-                  apply: Optional[Callable[[int, int], None]] = None, chunk: int = 0, order: int = 0) -> None:
+                  apply: Optional[Callable[[int, int], None]] = None, chunk: int = 0, order: int = 0,
+                  grad_again: Optional[Callable[[int, int], object]] = None) -> None:
     """Run one layer over this rank's `n_tokens` tokens.
 
     grad(t0, t1) -> G: gradient of the loss over local tokens [t0, t1) at the current weights.
@@ -28,6 +29,8 @@ def sharded_layer(n_tokens: int, steps: int, grad: Callable[[int, int], object],
     chunk > 0: causal carry over chunks of `chunk` local tokens (each chunk of the
     whole sequence is the union of the ranks' chunk c); order 0 applies before the
     chunk's update, order 1 after.  chunk = 0: one bidirectional chunk, apply after.
+    grad_again(t0, t1), if given, is used for the second and later inner steps of a
+    chunk: the same gradient, reusing what the first call prepared for those tokens.
     All ranks must pass the same n_tokens, chunk and steps so the collectives line up.
     """
     size = chunk if chunk > 0 else n_tokens
@@ -35,8 +38,8 @@ def sharded_layer(n_tokens: int, steps: int, grad: Callable[[int, int], object],
         c1 = min(n_tokens, c0 + size)
         if chunk > 0 and order == 0 and apply is not None:
             apply(c0, c1)
-        for _ in range(steps):
-            G = grad(c0, c1)
+        for st in range(steps):
+            G = grad(c0, c1) if st == 0 or grad_again is None else grad_again(c0, c1)
             allreduce(G)
             step(G)
         if chunk > 0 and order == 1 and apply is not None:

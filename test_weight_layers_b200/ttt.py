@@ -64,9 +64,12 @@ def lib() -> ctypes.CDLL:
             "ttt_l2norm": (I, [P, I64, Dims, I64, I, P]),
             "ttt_shortconv2d": (I, [P, I64, P, I64, P, I, I, I, I, I, I, P]),
             "ttt_grad": (I, [Weights, P, P, P, I64, Dims, ctypes.POINTER(IOCfg), I, P, P, SZ, P]),
+            "ttt_grad_prepared": (I, [Weights, P, P, P, I64, Dims, ctypes.POINTER(IOCfg), I, P, P, SZ, P]),
             "ttt_step": (I, [Weights, P, ctypes.POINTER(NSCfg), Dims, I, P, SZ, P]),
             "ttt_update": (I, [Weights, P, P, P, I64, I, ctypes.POINTER(NSCfg), Dims, ctypes.POINTER(IOCfg), I, P, SZ,
                                P]),
+            "ttt_update_conv": (I, [Weights, P, P, P, I64, I, ctypes.POINTER(NSCfg), P, I, I, I, Dims,
+                                    ctypes.POINTER(IOCfg), I, P, SZ, P]),
             "ttt_apply": (I, [Weights, P, P, I64, Dims, ctypes.POINTER(IOCfg), I, P, SZ, P]),
             "ttt_apply_noalloc": (I, [Weights, P, P, I64, Dims, ctypes.POINTER(IOCfg), I, P]),
             "ttt_chunked": (I, [Weights, P, P, P, P, P, I64, I64, I, I, ctypes.POINTER(NSCfg), Dims,
@@ -169,6 +172,13 @@ def ttt_grad(W: Weights, K, V, eta, T, dm: Dims, io: IOCfg, G, ws, stream=None):
                                       _ptr(G), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def ttt_grad_prepared(W: Weights, K, V, eta, T, dm: Dims, io: IOCfg, G, ws, stream=None):
+    """ttt_grad reusing the operands the last ttt_grad on `ws` prepared (same K, V, eta, T)."""
+    _check("ttt_grad_prepared", lib().ttt_grad_prepared(W, _ptr(K), _ptr(V), _ptr(eta), T, dm, ctypes.byref(io),
+                                                        dtype_code(K.dtype), _ptr(G), _ptr(ws), ws.numel(),
+                                                        _stream(stream)))
+
+
 def ttt_step(W: Weights, G, ns: NSCfg, dm: Dims, dtype: int, ws, stream=None):
     _check("ttt_step", lib().ttt_step(W, _ptr(G), ctypes.byref(ns), dm, dtype, _ptr(ws), ws.numel(), _stream(stream)))
 
@@ -177,6 +187,14 @@ def ttt_update(W: Weights, K, V, eta, T, steps, ns: NSCfg, dm: Dims, io: IOCfg, 
     _check("ttt_update", lib().ttt_update(W, _ptr(K), _ptr(V), _ptr(eta), T, steps, ctypes.byref(ns), dm,
                                           ctypes.byref(io), dtype_code(K.dtype), _ptr(ws), ws.numel(),
                                           _stream(stream)))
+
+
+def ttt_update_conv(W: Weights, K, V, eta, T, steps, ns: NSCfg, taps, grid_h, grid_w, dm: Dims, io: IOCfg, ws,
+                    act=0, stream=None):
+    """ttt_update on ShortConv2D(V), the conv folded into the update's operand preparation."""
+    _check("ttt_update_conv", lib().ttt_update_conv(W, _ptr(K), _ptr(V), _ptr(eta), T, steps, ctypes.byref(ns),
+                                                    _ptr(taps), grid_h, grid_w, act, dm, ctypes.byref(io),
+                                                    dtype_code(K.dtype), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def ttt_apply(W: Weights, Q, O, T, dm: Dims, io: IOCfg, ws, stream=None):

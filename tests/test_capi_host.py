@@ -166,3 +166,18 @@ def test_wide_head_shapes_are_accepted(lib):
     rc = lib.ttt_apply_noalloc(W, FAKE, ctypes.c_void_p(1 << 23), 10, T.dims(1, 256, 256),
                                ctypes.byref(T.io_cfg()), T.TTT_BF16, None)
     assert rc == T.TTT_ERR_UNSUPPORTED
+
+
+def test_update_conv_validation(lib):
+    d = T.dims(4, 192, 768)
+    W = T.Weights(1 << 20, 1 << 21, 1 << 22)
+    ns, io = T.ns_cfg(), T.io_cfg()
+    need = T.ttt_workspace_bytes(d, 2 * 37 * 37 + 1, T.TTT_BF16)
+    call = lambda T_, gh, gw, dt, act=0: lib.ttt_update_conv(W, FAKE, FAKE, FAKE, T_, 1, ctypes.byref(ns), FAKE, gh, gw,
+                                                            act, d, ctypes.byref(io), dt, FAKE, need, None)
+    assert call(2 * 37 * 37 + 1, 37, 37, T.TTT_BF16) == T.TTT_ERR_INVALID       # not whole frames
+    assert call(2 * 37 * 37, 37, 37, T.TTT_BF16, act=2) == T.TTT_ERR_INVALID    # act is 0 or 1
+    assert call(2 * 37 * 37, 0, 37, T.TTT_BF16) == T.TTT_ERR_INVALID
+    need32 = T.ttt_workspace_bytes(d, 2 * 37 * 37, T.TTT_FP32)
+    assert lib.ttt_update_conv(W, FAKE, FAKE, FAKE, 2 * 37 * 37, 1, ctypes.byref(ns), FAKE, 37, 37, 0, d,
+                               ctypes.byref(io), T.TTT_FP32, FAKE, need32, None) == T.TTT_ERR_UNSUPPORTED

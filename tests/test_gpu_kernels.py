@@ -139,6 +139,29 @@ def test_grad_is_deterministic(dt):
     assert torch.equal(G1, G2)
 
 
+@pytest.mark.parametrize("dt,d,m", [(T.TTT_BF16, 192, 256), (T.TTT_FP32, 64, 128), (T.TTT_BF16, 256, 512)])
+def test_grad_prepared_equals_grad_after_a_step(dt, d, m):
+    # the second inner step of the multi-device update: gradient, step, then the gradient
+    # at the new weights from the operands the first call prepared -- the same result
+    # as a fresh ttt_grad, bit for bit
+    dtype = torch.bfloat16 if dt == T.TTT_BF16 else torch.float32
+    H, T_ = 2, 700
+    W, K, V, eta = _grad_case(H, d, m, T_, dtype, seed=35)
+    dm = T.dims(H, d, m)
+    Kd, Vd, ed = K.cuda(), V.cuda(), eta.cuda()
+    ws = T.workspace(dm, T_, dt)
+    n = H * m * d
+    G = torch.empty((3 * n,), dtype=torch.float32, device="cuda")
+    T.ttt_grad(W.abi, Kd, Vd, ed, T_, dm, T.io_cfg(), G, ws)
+    T.ttt_step(W.abi, G, T.ns_cfg(), dm, dt, ws)
+    G2 = torch.full_like(G, float("nan"))
+    T.ttt_grad_prepared(W.abi, Kd, Vd, ed, T_, dm, T.io_cfg(), G2, ws)
+    G3 = torch.full_like(G, float("nan"))
+    T.ttt_grad(W.abi, Kd, Vd, ed, T_, dm, T.io_cfg(), G3, ws)
+    check_status(ws)
+    assert torch.equal(G2, G3)
+
+
 # bf16 shapes cover every Newton-Schulz path: one cluster launch with 192 rows and
 # 6 or 3 column blocks, with 128 rows and 2 or 1 blocks; per-product launches
 # for 192 x 320 (columns not a multiple of 128) and 64 x 128 (64 rows)
@@ -193,6 +216,37 @@ def test_step_matches_oracle_wide(H, d, m, iters, renorm, lr):
                                         f64(Gflat[2 * n:].reshape(H, d, m))), cfg)
     errs = weight_errors(W.oracle(), ref)
     assert max(errs) < 1e-4, errs
+
+
+@pytest.mark.parametrize("H,d,m,N,gh,gw,act", [(2, 192, 256, 3, 5, 7, 0), (2, 128, 128, 2, 9, 4, 1),
+                                                (1, 256, 256, 2, 6, 6, 0), (4, 192, 768, 4, 37, 37, 0)])
+def test_update_conv_matches_conv_then_update(H, d, m, N, gh, gw, act):
+    # ShortConv2D folded into the update's preparation: the same update as ttt_shortconv2d
+    # followed by ttt_update (only the rounding of V' differs: once to fp16 instead of
+    # bf16 then fp16), and within the layer tolerance of the oracle
+    T_ = N * gh * gw
+    g = torch.Generator().manual_seed(60 + d)
+    K = rand_tokens(T_, H, d, torch.bfloat16, 61)
+    V = rand_tokens(T_, H, d, torch.bfloat16, 62)
+    eta = rand_eta(T_, H, 63, scale=0.01)
+    taps = torch.randn((H * d, 3, 3), generator=g) / 3
+    dm = T.dims(H, d, m)
+    ns = T.ns_cfg()
+    W1 = DevWeights(*rand_weights(H, d, m, 64))
+    W2 = DevWeights(*rand_weights(H, d, m, 64))
+    W0 = W1.oracle()
+    ws = T.workspace(dm, T_, T.TTT_BF16)
+    Kd, Vd, ed, td = K.cuda(), V.cuda(), eta.cuda(), taps.cuda()
+    T.ttt_update_conv(W1.abi, Kd, Vd, ed, T_, 2, ns, td, gh, gw, dm, T.io_cfg(), ws, act=act)
+    check_status(ws)
+    Vc = torch.empty_like(Vd)
+    T.ttt_shortconv2d(Vd, Vc, td, N, gh, gw, H * d, act)
+    T.ttt_update(W2.abi, Kd, Vc, ed, T_, 2, ns, dm, T.io_cfg(), ws)
+    check_status(ws)
+    assert max(weight_errors(W1.oracle(), W2.oracle())) < 1e-2
+    ref = O.update(W0, f64(K), f64(V), f64(eta), 2, O.NSConfig(), conv=(taps.double().numpy(), N, gh, gw, act))
+    errs = weight_errors(W1.oracle(), ref)
+    assert max(errs) < TOL_BF16, errs
 
 
 def test_update_eta_zero_keeps_weights_bf16():
