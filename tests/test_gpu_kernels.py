@@ -163,10 +163,11 @@ def test_grad_prepared_equals_grad_after_a_step(dt, d, m):
 
 
 # bf16 shapes cover every Newton-Schulz path: one cluster launch with 192 rows and
-# 6 or 3 column blocks, with 128 rows and 2 or 1 blocks; per-product launches
+# 6, 3 or 2 column blocks, with 128 rows and 2 or 1 blocks; per-product launches
 # for 192 x 320 (columns not a multiple of 128) and 64 x 128 (64 rows)
 @pytest.mark.parametrize("dt,d,m", [(T.TTT_BF16, 192, 768), (T.TTT_BF16, 192, 384), (T.TTT_BF16, 128, 256),
-                                    (T.TTT_BF16, 128, 128), (T.TTT_BF16, 192, 320), (T.TTT_BF16, 128, 64),
+                                    (T.TTT_BF16, 128, 128), (T.TTT_BF16, 192, 256), (T.TTT_BF16, 192, 320),
+                                    (T.TTT_BF16, 128, 64),
                                     (T.TTT_FP32, 64, 128), (T.TTT_FP32, 96, 32)])
 @pytest.mark.parametrize("iters,renorm,lr", [(5, 1, 1.0), (0, 0, 0.01), (3, 0, 0.5), (1, 1, 1.0)])
 def test_step_matches_oracle(dt, d, m, iters, renorm, lr):
