@@ -34,7 +34,7 @@ def _data(H=2, d=6, m=8, T=48, seed=7):
     return W, K, V, Q, eta
 
 
-def _rank_main(rank, world, port, chunk, steps, order, out_q):
+def _rank_main(rank, world, port, chunk, steps, order, again, out_q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -46,11 +46,20 @@ def _rank_main(rank, world, port, chunk, steps, order, out_q):
         H, d, m = W.dims
         cfg = O.NSConfig()
         state = {"W": W}
+        calls = {"grad": 0, "again": 0}
         outs = np.zeros((per, H * d))
 
-        def grad(t0, t1):
+        def grad_of(t0, t1):
             g = O.grad(state["W"], O.l2norm_heads(Kl[t0:t1], H, d), Vl[t0:t1], el[t0:t1])
             return torch.from_numpy(np.concatenate([g.W1.ravel(), g.W3.ravel(), g.W2.ravel()]))
+
+        def grad(t0, t1):
+            calls["grad"] += 1
+            return grad_of(t0, t1)
+
+        def grad_again(t0, t1):
+            calls["again"] += 1
+            return grad_of(t0, t1)
 
         def allreduce(G):
             dist.all_reduce(G)
@@ -64,25 +73,33 @@ def _rank_main(rank, world, port, chunk, steps, order, out_q):
         def apply(t0, t1):
             outs[t0:t1] = O.apply(state["W"], Ql[t0:t1])
 
-        sharded_layer(per, steps, grad, allreduce, step, apply, chunk=chunk, order=order)
+        sharded_layer(per, steps, grad, allreduce, step, apply, chunk=chunk, order=order,
+                      grad_again=grad_again if again else None)
         Wf = state["W"]
-        out_q.put((rank, np.concatenate([Wf.W1.ravel(), Wf.W3.ravel(), Wf.W2.ravel()]), outs))
+        out_q.put((rank, np.concatenate([Wf.W1.ravel(), Wf.W3.ravel(), Wf.W2.ravel()]), outs, calls))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("chunk,steps,order", [(0, 1, 0), (0, 2, 0), (8, 1, 0), (8, 1, 1)])
-def test_two_rank_gcs_equals_single_process(chunk, steps, order):
+# again: the later inner steps of a chunk go through grad_again (the library's
+# ttt_grad_prepared, which reuses the operands the chunk's first ttt_grad prepared)
+@pytest.mark.parametrize("chunk,steps,order,again", [(0, 1, 0, False), (0, 2, 0, False), (8, 1, 0, False),
+                                                     (8, 1, 1, False), (0, 2, 0, True), (8, 2, 1, True)])
+def test_two_rank_gcs_equals_single_process(chunk, steps, order, again):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, chunk, steps, order, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, chunk, steps, order, again, q)) for r in range(2)]
     for p in procs:
         p.start()
     res = {}
     for _ in range(2):
-        r, w, o = q.get(timeout=120)
+        r, w, o, calls = q.get(timeout=120)
         res[r] = (w, o)
+        # one first-step gradient per chunk; the later steps through grad_again when given
+        n_chunks = 1 if chunk == 0 else (len(_data()[1]) // 2) // chunk
+        later = n_chunks * (steps - 1)
+        assert calls == ({"grad": n_chunks, "again": later} if again else {"grad": n_chunks + later, "again": 0})
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
