@@ -38,8 +38,9 @@ METRIC = "TTT-layer tokens/sec (update+apply) and % of B200 bf16 tensor peak"
 UNIT = "tokens/s"
 L2_BYTES = 126 << 20
 L2_FLUSH_BYTES = 512 << 20
-UPDATE_OPERANDS = ("fp16 tensor-core operands: K^ (normalised), V' = -2^8 eta v (one rounding), fast-weight copy, "
-                   "dH and u (fp32 accumulation)")
+UPDATE_OPERANDS = ("fp16 tensor-core operands: K^ (normalised), V' = -s eta v with a per-call power-of-two s "
+                   "(s max|eta| in [16, 32); one rounding), fast-weight copy, dH and u (fp32 accumulation); "
+                   "out-of-range operands are reported as TTT_ERR_RANGE and leave W unchanged")
 
 
 def parse():

@@ -44,8 +44,9 @@
  *    fp16 intermediates in the workspace); TTT_FP32 mode runs fp32 CUDA-core
  *    kernels for any d <= 256 and m a multiple of 32.  Other shapes return
  *    TTT_ERR_UNSUPPORTED.
- *  - Operand range of the TTT_BF16 update (ttt_grad, ttt_update, ttt_chunked,
- *    ttt_layer_host).  The gradient GEMMs run on fp16 operands with fp32
+ *  - Operand range of the TTT_BF16 update (ttt_grad, ttt_grad_prepared,
+ *    ttt_update, ttt_update_conv, ttt_chunked, ttt_layer_host).  The gradient
+ *    GEMMs run on fp16 operands with fp32
  *    accumulation: k^ (k / ||k|| with qk_l2norm = 1, else k itself),
  *    V' = -s eta v with a power of two s chosen per call so that
  *    s * max|eta| lies in [16, 32) (for ttt_layer_host with chunk = 0: one s
@@ -173,7 +174,8 @@ int ttt_update(ttt_weights W, const void* K, const void* V, const float* eta, in
  * operand, instead of first to bf16 -- V' itself is never written.  taps: device
  * float [H*d][3][3].  TTT_BF16 only; T must be whole frames; the head dim d must be
  * a multiple of 64 and a frame row must fit a shared-memory band (true for grids up
- * to several hundred tokens wide), else TTT_ERR_UNSUPPORTED. */
+ * to several hundred tokens wide), else TTT_ERR_UNSUPPORTED.  The operand range of
+ * the update (above) applies to the convolved values in place of V. */
 int ttt_update_conv(ttt_weights W, const void* K, const void* V, const float* eta, int64_t T, int steps,
                     const ttt_ns_cfg* ns, const float* taps, int grid_h, int grid_w, int act, ttt_dims dims,
                     const ttt_io_cfg* io, ttt_dtype dtype, void* ws, size_t ws_bytes, void* stream);

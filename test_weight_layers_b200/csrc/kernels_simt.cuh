@@ -832,9 +832,11 @@ __global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, fl
   const int64_t n = (int64_t)m * d;
   const float sc = 1.0f / (sqrtf(sum_parts(parts + b * NORM_PARTS)) + eps);
   const float* g = G + (int64_t)b * n;
-  // the copy with G's layout: X (wide) or XT (tall); the transposed copy: the other
-  float* same = (tall ? XT : X) + (int64_t)b * n;
-  float* trans = (tall ? X : XT) + (int64_t)b * n;
+  // the copy with G's layout: X (wide) or XT (tall); the transposed copy: the
+  // other.  XT == nullptr: only X is written (the tensor-core iterations never
+  // read XT).
+  float* same = tall ? (XT ? XT + (int64_t)b * n : nullptr) : X + (int64_t)b * n;
+  float* trans = tall ? X + (int64_t)b * n : (XT ? XT + (int64_t)b * n : nullptr);
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   if (r0 >= R || c0 >= C) return;
   for (int yy = threadIdx.y; yy < 32; yy += 8) {
@@ -842,10 +844,11 @@ __global__ void k_ns_init(const float* __restrict__ G, float* __restrict__ X, fl
     float v = 0.f;
     if (r < R && c < C) {
       v = g[(int64_t)r * C + c] * sc;
-      same[(int64_t)r * C + c] = v;
+      if (same) same[(int64_t)r * C + c] = v;
     }
     tile[yy][threadIdx.x] = v;
   }
+  if (!trans) return;
   __syncthreads();
   for (int yy = threadIdx.y; yy < 32; yy += 8) {
     const int c = c0 + yy, r = r0 + threadIdx.x;  // trans is (C x R)

@@ -970,8 +970,8 @@ int run_ns_step(const ttt_weights& W, const float* G, const ttt_ns_cfg& ns, cons
   if (ns.iters > 0) {
     k_frob_partials<<<dim3(nb, NORM_PARTS), 256, 0, s>>>(G, n, w.norms);
     TTT_LAUNCHED();
-    TTT_TRY(launch_pdl(k_ns_init, dim3((c + 31) / 32, (c + 31) / 32, nb), dim3(32, 8), 0, s, G, w.X, w.XT,
-                       (const float*)w.norms, H, dd, mm, ns.eps));
+    TTT_TRY(launch_pdl(k_ns_init, dim3((c + 31) / 32, (c + 31) / 32, nb), dim3(32, 8), 0, s, G, w.X,
+                       dt == TTT_BF16 ? (float*)nullptr : w.XT, (const float*)w.norms, H, dd, mm, ns.eps));
     float *X = w.X, *X2 = w.X2, *XT = w.XT, *XT2 = w.XT2;
     if (dt == TTT_BF16) {
       if (ns_cluster_usable(r, c)) {
