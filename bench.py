@@ -442,7 +442,7 @@ def run_ours(args, cfg):
         roof = {"bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
                 "frac_of_burst": ach / peaks["bf16_tflops"], "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
                 "traffic": None if wide else traffic_per_launch(tok_per_launch),
-                "kernel": ("k_wgemm gradient products with k_prep_wide (2-SM pairs)" if wide else "k_update_grad_tc"),
+                "kernel": ("k_wgemm gradient products on 2-SM pairs: Z, [H1|H3] with the SwiGLU backward, weight gradients" if wide else "k_update_grad_tc"),
                 "peak_kind": "fp16/bf16 dense (same tensor rate), " + peak_kind,
                 "launch_ms": g_ms / g_n}
     elif g_n:
