@@ -438,6 +438,11 @@ struct ApLayout {
 };
 
 constexpr int AP_THREADS = 352;  // warp 0: Q + W1|W3 TMA, 1: MMA, 2..9: epilogue, 10: W2 TMA
+// O of chunk c is issued after H of chunk c + AP_OLAG: the epilogue has that many
+// H products' time to turn H_c into P_c before the tensor pipe needs it (H is
+// double-buffered in TMEM and the epilogue drains H_c first, so H_(c+2) may
+// already overwrite it)
+constexpr int AP_OLAG = 2;
 
 // Fused SwiGLU apply on 2-SM tensor-core pairs (cta_group::2).  A cluster of two
 // CTAs owns a 256-token tile (128 per CTA) of one head; every MMA is M = 256:
@@ -617,10 +622,12 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
           __syncwarp();
           p13 ^= (s13 == L::NS13 - 1) ? 1u : 0u;
           s13 = (s13 == L::NS13 - 1) ? 0u : s13 + 1;
-          if (c > 0 && !do_o(gc - 1, c == 1, it)) { ok = false; break; }
+          if (c >= AP_OLAG && !do_o(gc - AP_OLAG, c == AP_OLAG, it)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!do_o(gc - 1, nc == 1, it)) break;
+        // the item's last O products
+        for (int j = nc > AP_OLAG ? nc - AP_OLAG : 0; ok && j < nc; ++j) ok = do_o(gc - nc + j, j == 0, it);
+        if (!ok) break;
         if (el) umma_commit_pair(odone);
         __syncwarp();
       }
