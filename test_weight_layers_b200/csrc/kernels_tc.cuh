@@ -473,14 +473,14 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* qfull = bars + 0;              // leader: TMA bytes of both CTAs
-  uint64_t* qfree = bars + 1;              // both: MMA done reading Q (1) + this CTA's epilogue read its norms (256)
+  uint64_t* qfree = bars + 1;              // both: MMA done reading Q (1) + this CTA's epilogue read its norms
   uint64_t* w13full = bars + 2;            // [NS13] leader
   uint64_t* w13free = w13full + L::NS13;   // [NS13] both
   uint64_t* w2full = w13free + L::NS13;    // [NS2] leader
   uint64_t* w2free = w2full + L::NS2;      // [NS2] both
   uint64_t* hfull = w2free + L::NS2;       // [2] both
-  uint64_t* hfree = hfull + 2;             // [2] leader: 512 arrivals (both epilogues)
-  uint64_t* pfull = hfree + 2;             // [2] leader: 512 arrivals
+  uint64_t* hfree = hfull + 2;             // [2] leader: 256 arrivals (a chunk's epilogue group, both CTAs)
+  uint64_t* pfull = hfree + 2;             // [2] leader: 256 arrivals
   uint64_t* pfree = pfull + 2;             // [2] both
   uint64_t* odone = pfree + 2;             // both
   uint64_t* ofree = odone + 1;             // leader: 512 arrivals
@@ -488,7 +488,9 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
-    mbar_init(qfree, 1 + 256);
+    // the MMAs' commit, and every epilogue warp that handles a chunk of the item (one
+    // group of four when the item has a single chunk, else both)
+    mbar_init(qfree, 1 + (nc >= 2 ? 256 : 128));
     for (int i = 0; i < L::NS13; ++i) {
       mbar_init(w13full + i, 1);
       mbar_init(w13free + i, 1);
@@ -499,8 +501,8 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(hfull + i, 1);
-      mbar_init(hfree + i, 512);
-      mbar_init(pfull + i, 512);
+      mbar_init(hfree + i, 256);  // one epilogue group (4 warps) of each CTA per chunk
+      mbar_init(pfull + i, 256);
       mbar_init(pfree + i, 1);
     }
     mbar_init(odone, 1);
@@ -633,9 +635,12 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
       }
     }
   } else {
-    // ---------------- epilogue warps 2..9 (both CTAs)
+    // ---------------- epilogue warps 2..9 (both CTAs): two groups of four warps
+    // take alternate chunks (group = chunk parity = H buffer), so one group turns
+    // H_c into P_c while the other drains H_(c+1); each warp covers its 32 TMEM
+    // lanes (token rows) and all 64 columns of the chunk, 32 at a time
     const int q = warp & 3;
-    const int ch = (warp - 2) >> 2;
+    const int ch = (warp - 2) >> 2;  // this warp's group; also its half of O's columns
     const int row = q * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const uint32_t hfree_l0 = cluster_addr(hfree, 0), hfree_l1 = cluster_addr(hfree + 1, 0);
@@ -646,13 +651,16 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     for (int item = pair; ok && item < n_items; item += npairs, ++it) {
       const int tile = item / H, h = item % H;
       float r = 1.f;
+      bool first = true;  // this group's first chunk of the item
       for (int c = 0; c < nc; ++c, ++gc) {
         const int hb = gc & 1;
+        if (hb != ch) continue;  // the other group's chunk
         if (!__all_sync(0xffffffffu, mbar_wait(hfull + hb, (gc >> 1) & 1, g))) { ok = false; break; }
         tc_fence_after();
-        if (c == 0) {
-          // The first H of the item has read the query tile, so it is in shared
-          // memory; it stays there until this CTA's epilogue releases it (qfree).
+        if (first) {
+          first = false;
+          // The item's first H has read the query tile, so it is in shared
+          // memory; it stays there until both groups' epilogues release it (qfree).
           // q^ = q / max(||q||, 1e-12): the GEMM used the raw query, so the
           // inverse norm scales H1 and H3 rows here (rows past T were zero-filled).
           if (qnorm) {
@@ -675,27 +683,32 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_n(qfree, 32);
         }
-        uint32_t a1[32], a3[32];
-        tmem_ld32(tmem + lane_base + L::H_COL + hb * 128 + ch * 32, a1);
-        tmem_ld32(tmem + lane_base + L::H_COL + hb * 128 + 64 + ch * 32, a3);
-        tmem_ld_wait(a1);
-        tmem_ld_wait(a3);
-        tc_fence_before();
-        warp_arrive_cluster(hb ? hfree_l1 : hfree_l0);
-        uint32_t pk[16];
+        uint32_t pk[2][16];
         const float2 r2 = make_float2(r, r);
         const float2 half2 = make_float2(0.5f, 0.5f);
-        // sigmoid(h1) = 1/2 + tanh(h1/2)/2 with tanh in half precision (two per
-        // MUFU operation): its error (~2^-11) is well below the bf16 rounding of P
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 h1 = __fmul2_rn(make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1])), r2);
-          const float2 h3 = __fmul2_rn(make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1])), r2);
-          const float2 hh = __fmul2_rn(h1, half2);
-          const float2 th = unpack_f16x2(tanh_f16x2(pack_f16x2(hh.x, hh.y)));
-          const float2 sg = __ffma2_rn(th, half2, half2);
-          const float2 pv = __fmul2_rn(__fmul2_rn(h1, sg), h3);  // SiLU(h1) * h3
-          pk[j >> 1] = pack_bf16x2(pv.x, pv.y);
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t a1[32], a3[32];
+          tmem_ld32(tmem + lane_base + L::H_COL + hb * 128 + hc * 32, a1);
+          tmem_ld32(tmem + lane_base + L::H_COL + hb * 128 + 64 + hc * 32, a3);
+          tmem_ld_wait(a1);
+          tmem_ld_wait(a3);
+          if (hc == 1) {
+            tc_fence_before();
+            warp_arrive_cluster(hb ? hfree_l1 : hfree_l0);
+          }
+          // sigmoid(h1) = 1/2 + tanh(h1/2)/2 with tanh in half precision (two per
+          // MUFU operation): its error (~2^-11) is well below the bf16 rounding of P
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 h1 = __fmul2_rn(make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1])), r2);
+            const float2 h3 = __fmul2_rn(make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1])), r2);
+            const float2 hh = __fmul2_rn(h1, half2);
+            const float2 th = unpack_f16x2(tanh_f16x2(pack_f16x2(hh.x, hh.y)));
+            const float2 sg = __ffma2_rn(th, half2, half2);
+            const float2 pv = __fmul2_rn(__fmul2_rn(h1, sg), h3);  // SiLU(h1) * h3
+            pk[hc][j >> 1] = pack_bf16x2(pv.x, pv.y);
+          }
         }
         if (gc >= 2 && !__all_sync(0xffffffffu, mbar_wait(pfree + hb, ((gc >> 1) - 1) & 1, g))) {
           ok = false;
@@ -703,9 +716,11 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
         }
         uint8_t* sp = smem + L::P_OFF + hb * TC_BLK;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          *reinterpret_cast<uint4*>(sp + sw128_offset(row, ch * 4 + cc)) =
-              make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+        for (int hc = 0; hc < 2; ++hc)
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+            *reinterpret_cast<uint4*>(sp + sw128_offset(row, hc * 4 + cc)) =
+                make_uint4(pk[hc][4 * cc], pk[hc][4 * cc + 1], pk[hc][4 * cc + 2], pk[hc][4 * cc + 3]);
         fence_async_smem();
         warp_arrive_cluster(hb ? pfull_l1 : pfull_l0);
       }
