@@ -697,14 +697,15 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
             tc_fence_before();
             warp_arrive_cluster(hb ? hfree_l1 : hfree_l0);
           }
-          // sigmoid(h1) = 1/2 + tanh(h1/2)/2 with tanh in half precision (two per
-          // MUFU operation): its error (~2^-11) is well below the bf16 rounding of P
+          // sigmoid(h1) = 1/2 + tanh(h1/2)/2, tanh.approx.f32 (one MUFU operation per
+          // element; the half-precision pair form saves MUFU work but its three
+          // conversions per pair cost more: 2.93 vs 2.86 ms in a same-process A/B)
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             const float2 h1 = __fmul2_rn(make_float2(__uint_as_float(a1[j]), __uint_as_float(a1[j + 1])), r2);
             const float2 h3 = __fmul2_rn(make_float2(__uint_as_float(a3[j]), __uint_as_float(a3[j + 1])), r2);
             const float2 hh = __fmul2_rn(h1, half2);
-            const float2 th = unpack_f16x2(tanh_f16x2(pack_f16x2(hh.x, hh.y)));
+            const float2 th = make_float2(tanh_approx(hh.x), tanh_approx(hh.y));
             const float2 sg = __ffma2_rn(th, half2, half2);
             const float2 pv = __fmul2_rn(__fmul2_rn(h1, sg), h3);  // SiLU(h1) * h3
             pk[hc][j >> 1] = pack_bf16x2(pv.x, pv.y);
