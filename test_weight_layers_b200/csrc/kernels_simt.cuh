@@ -205,7 +205,10 @@ __device__ __forceinline__ void store16_h(__half* p, const float (&v)[8]) {
   *reinterpret_cast<uint4*>(p) = x;
 }
 
-__global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restrict__ K, int64_t ldk,
+// RN: 16-byte vectors per lane of a row (H*d <= 256 RN); more than 4 takes the
+// per-head loop
+template <int RN>
+__global__ void __launch_bounds__(256, RN <= 3 ? 3 : 2) k_prep_kv(const __nv_bfloat16* __restrict__ K, int64_t ldk,
                                                     const __nv_bfloat16* __restrict__ V, int64_t ldv,
                                                     const float* __restrict__ eta,
                                                     const float* __restrict__ eta_part,
@@ -220,32 +223,46 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int HD = H * d;
   const int nvt = HD / VN;
-  for (int64_t t = warp_id; t < rows; t += nwarps) {
-    const __nv_bfloat16* krow = K + t * ldk;
-    const __nv_bfloat16* vrow = V + t * ldv;
-    if (nvt <= 32 * RN_MAX_VEC) {
-      // the row stays packed (bf16) in registers: small footprint, many tokens in flight per SM
-      uint4 xk[RN_MAX_VEC], xv[RN_MAX_VEC];
-      int hv[RN_MAX_VEC];
-      // eta of this token: lane h < H holds head h's weight (one load per token,
-      // issued with the row loads); the vectors fetch theirs by shuffle
-      const float eh = (lane < H) ? __ldg(eta + t * H + lane) : 0.f;
+  if (nvt <= 32 * RN) {
+    // The row stays packed (bf16) in registers: small footprint, many tokens in
+    // flight per SM.  The next token's row is loaded while this one is
+    // converted, so a warp always has a row's loads outstanding.
+    int hv[RN];  // head of this lane's k-th vector (-1: past the row)
 #pragma unroll
-      for (int k = 0; k < RN_MAX_VEC; ++k) {
+    for (int k = 0; k < RN; ++k) {
+      const int v = lane + 32 * k;
+      hv[k] = v < nvt ? v * VN / d : -1;
+    }
+    // eta of a token: lane h < H holds head h's weight (one load per token,
+    // issued with the row loads); the vectors fetch theirs by shuffle
+    auto load_row = [&](int64_t t, uint4 (&xk)[RN], uint4 (&xv)[RN], float& eh) {
+      const __nv_bfloat16* krow = K + t * ldk;
+      const __nv_bfloat16* vrow = V + t * ldv;
+      eh = (lane < H) ? __ldg(eta + t * H + lane) : 0.f;
+#pragma unroll
+      for (int k = 0; k < RN; ++k) {
         const int v = lane + 32 * k;
-        hv[k] = v < nvt ? v * VN / d : -1;
         if (hv[k] >= 0) {
           xk[k] = __ldg(reinterpret_cast<const uint4*>(krow + v * VN));
           xv[k] = Vh ? __ldg(reinterpret_cast<const uint4*>(vrow + v * VN)) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      float inv[RN_MAX_VEC];
+    };
+    uint4 xk[RN], xv[RN];
+    float eh = 0.f;
+    int64_t t = warp_id;
+    if (t < rows) load_row(t, xk, xv, eh);
+    for (; t < rows; t += nwarps) {
+      uint4 nk[RN], nv[RN];
+      float ne = 0.f;
+      if (t + nwarps < rows) load_row(t + nwarps, nk, nv, ne);
+      float inv[RN];
 #pragma unroll
-      for (int k = 0; k < RN_MAX_VEC; ++k) inv[k] = 1.f;
+      for (int k = 0; k < RN; ++k) inv[k] = 1.f;
       if (l2norm) {
-        float ss[RN_MAX_VEC];
+        float ss[RN];
 #pragma unroll
-        for (int k = 0; k < RN_MAX_VEC; ++k) {
+        for (int k = 0; k < RN; ++k) {
           ss[k] = 0.f;
           if (hv[k] >= 0) {
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&xk[k]);
@@ -259,16 +276,16 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
         for (int h = 0; h < H; ++h) {
           float p = 0.f;
 #pragma unroll
-          for (int k = 0; k < RN_MAX_VEC; ++k) p += (hv[k] == h) ? ss[k] : 0.f;
+          for (int k = 0; k < RN; ++k) p += (hv[k] == h) ? ss[k] : 0.f;
           p = warp_sum(p);
           const float r = 1.0f / fmaxf(sqrtf(p), 1e-12f);
 #pragma unroll
-          for (int k = 0; k < RN_MAX_VEC; ++k)
+          for (int k = 0; k < RN; ++k)
             if (hv[k] == h) inv[k] = r;
         }
       }
 #pragma unroll
-      for (int k = 0; k < RN_MAX_VEC; ++k) {
+      for (int k = 0; k < RN; ++k) {
         const float vek = vscale * __shfl_sync(0xffffffffu, eh, hv[k] >= 0 ? hv[k] : 0);
         if (hv[k] >= 0) {
           const __nv_bfloat162* hk = reinterpret_cast<const __nv_bfloat162*>(&xk[k]);
@@ -286,7 +303,17 @@ __global__ void __launch_bounds__(256, 4) k_prep_kv(const __nv_bfloat16* __restr
           if (Vh) *reinterpret_cast<uint4*>(Vh + t * HD + (lane + 32 * k) * VN) = ov;
         }
       }
-    } else {
+#pragma unroll
+      for (int k = 0; k < RN; ++k) {
+        xk[k] = nk[k];
+        xv[k] = nv[k];
+      }
+      eh = ne;
+    }
+  } else {
+    for (int64_t t = warp_id; t < rows; t += nwarps) {
+      const __nv_bfloat16* krow = K + t * ldk;
+      const __nv_bfloat16* vrow = V + t * ldv;
       for (int h = 0; h < H; ++h) {
         float ss = 0.f;
         for (int v = lane; v < d / VN; v += 32) {

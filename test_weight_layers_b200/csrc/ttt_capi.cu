@@ -473,8 +473,13 @@ int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, const
   if (T == 0) return TTT_OK;
   ProfScope ps(TTT_PROF_NORM, s);
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 16));
-  k_prep_kv<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, w.etapart, kh,
-                                   vh, T, d.heads, d.d, l2norm);
+  const int nvt = d.heads * d.d / 8;  // 16-byte vectors per row
+  if (nvt <= 96)
+    k_prep_kv<3><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, w.etapart,
+                                        kh, vh, T, d.heads, d.d, l2norm);
+  else
+    k_prep_kv<4><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, w.etapart,
+                                        kh, vh, T, d.heads, d.d, l2norm);
   TTT_LAUNCHED();
   return TTT_OK;
 }
