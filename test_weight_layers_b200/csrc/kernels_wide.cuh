@@ -38,8 +38,12 @@ struct WgLayout {
   static constexpr int A_OFF = 0;
   static constexpr int B_OFF = WG_STAGES * WG_HALF;
   static constexpr int BAR_OFF = 2 * WG_STAGES * WG_HALF;
-  static constexpr int BYTES = BAR_OFF + 256;
+  static constexpr int TB_ROW = 80;                  // a staged row: 32 16-bit values + 16 bytes of padding
+  static constexpr int TB_WARP = 32 * TB_ROW;        // one epilogue warp's 32 rows
+  static constexpr int TB_OFF = BAR_OFF + 256;       // 8 epilogue warps' staging buffers
+  static constexpr int BYTES = TB_OFF + 8 * TB_WARP;
   static constexpr int ALLOC = BYTES + 1024;
+  static constexpr int ALLOC_NO_TB = TB_OFF + 1024;  // epilogues that stage no rows
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
 
@@ -52,6 +56,15 @@ enum WgEpi : int {
   WG_GATE = 5,         // acc = o' W_g^T: out = o' rinv SiLU(acc) (bf16)
   WG_NSOUT = 6         // Newton-Schulz product: C = alpha acc + beta Cin (fp32) and its bf16 hi/lo parts
 };
+
+// dynamic shared memory of an instance: the row-staging buffers only where the
+// epilogue stores 16-bit rows through them
+template <int EPI>
+constexpr int wg_smem_bytes() {
+  return (EPI == WG_STORE16 || EPI == WG_STORE_BF16 || EPI == WG_SWIGLU_BWD || EPI == WG_SWIGLU_FWD)
+             ? WgLayout::ALLOC
+             : WgLayout::ALLOC_NO_TB;
+}
 
 // Everything a launch needs besides the tensor maps.  Items are
 // (split, mat, head, tm, tn) with tn fastest, so pairs running side by side
@@ -152,6 +165,26 @@ __device__ __forceinline__ float silu_f(float x) {
   float t;
   asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
   return x * fmaf(t, 0.5f, 0.5f);
+}
+
+// A warp's 32 rows x 32 16-bit columns (lane = row, four 16-byte vectors each) to
+// global memory with coalesced stores: the rows go through the warp's staging
+// buffer and leave as 8 rows x 64 contiguous bytes per store instruction, instead
+// of 32 rows x 16 bytes (32 cache lines per instruction).  g0: the first row's
+// first column; ldb: row stride in bytes; rows at or past nrows are not written.
+__device__ __forceinline__ void warp_rows_out(uint8_t* tb, const uint4 (&v)[4], uint8_t* g0, int64_t ldb,
+                                              int nrows) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();  // the previous use of the buffer has been read
+#pragma unroll
+  for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(tb + lane * WgLayout::TB_ROW + c * 16) = v[c];
+  __syncwarp();
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int r = s * 8 + (lane >> 2), c = lane & 3;
+    const uint4 x = *reinterpret_cast<const uint4*>(tb + r * WgLayout::TB_ROW + c * 16);
+    if (r < nrows) *reinterpret_cast<uint4*>(g0 + r * ldb + c * 16) = x;
+  }
 }
 
 // 8 consecutive fp16 / bf16 values from global memory as floats
@@ -322,6 +355,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
     // quarter q (32 output rows) and half of the tile's columns
     const int q = warp & 3, half = (warp - 2) >> 2;
     const int rloc = q * 32 + lane;  // row within this CTA's 128
+    uint8_t* tbuf = smem + WgLayout::TB_OFF + (warp - 2) * WgLayout::TB_WARP;  // this warp's staging rows
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const uint32_t accempty_l0 = cluster_addr(bars.accempty, 0), accempty_l1 = cluster_addr(bars.accempty + 1, 0);
     float scale = 1.f;
@@ -352,6 +386,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
       // the epilogue's own global inputs do not depend on the MMAs: their loads are issued
       // before waiting for the accumulator so their latency overlaps the wait
       uint4 pre[16], pre_z[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) pre_z[c] = make_uint4(0u, 0u, 0u, 0u);
       if (EPI == WG_SWIGLU_BWD) {
 #pragma unroll
         z_load(item, pre_z);
@@ -375,8 +411,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         for (int p = 0; p < 4; ++p) tmem_ld_wait(v[p]);
         tc_fence_before();
         warp_arrive_cluster(accempty_l);
-        if (row >= a.M) continue;
         if constexpr (EPI == WG_PARTIAL) {
+          if (row >= a.M) continue;
           // partial[s][mat][h][M][N] (g1, g3: [m][d]; g2: [d][m]), scaled by 1/s
           const int Nn = it.mat == 2 ? a.m : a.d;
           const int64_t n = (int64_t)a.m * a.d;
@@ -390,9 +426,13 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                   make_float4(__uint_as_float(v[p][c]) * scale, __uint_as_float(v[p][c + 1]) * scale,
                               __uint_as_float(v[p][c + 2]) * scale, __uint_as_float(v[p][c + 3]) * scale);
         } else {
+          // 32-column groups leave through the warp's staging buffer (coalesced)
           const int64_t col = (int64_t)it.h * a.out_head + it.tn * 256 + half * 128;
+          const int64_t row0 = row - lane;
+          const int nrows = (int)max((int64_t)0, min((int64_t)32, a.M - row0));
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
+            uint4 o[4];
 #pragma unroll
             for (int c = 0; c < 32; c += 8) {
               uint32_t w4[4];
@@ -401,16 +441,20 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                 w4[i] = EPI == WG_STORE16
                             ? pack_f16x2(__uint_as_float(v[p][c + 2 * i]), __uint_as_float(v[p][c + 2 * i + 1]))
                             : pack_bf16x2(__uint_as_float(v[p][c + 2 * i]), __uint_as_float(v[p][c + 2 * i + 1]));
-              uint8_t* dst = static_cast<uint8_t*>(a.out) + (row * a.ldo + col + p * 32 + c) * 2;
-              *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              o[c >> 3] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
+            warp_rows_out(tbuf, o, static_cast<uint8_t*>(a.out) + (row0 * a.ldo + col + p * 32) * 2, a.ldo * 2,
+                          nrows);
           }
         }
       } else if constexpr (EPI == WG_SWIGLU_BWD || EPI == WG_SWIGLU_FWD) {
         // m columns [tn*128 + half*64, +64) of head h, in two 32-column phases: H1 from
-        // accumulator columns half*64 + .., H3 from 128 + half*64 + ..
+        // accumulator columns half*64 + .., H3 from 128 + half*64 + ..; each phase's
+        // 32 x 32 outputs per warp leave through the staging buffer (coalesced)
         const int64_t col = (int64_t)it.h * a.m + it.tn * 128 + half * 64;
         const float r = (EPI == WG_SWIGLU_FWD && a.rvec && row < a.M) ? a.rvec[row * a.heads + it.h] : 1.f;
+        const int64_t row0 = row - lane;  // this warp's first row
+        const int nrows = (int)max((int64_t)0, min((int64_t)32, a.M - row0));
 #pragma unroll
         for (int ph = 0; ph < 2; ++ph) {
           uint32_t v1[32], v3[32];
@@ -422,7 +466,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
             tc_fence_before();
             warp_arrive_cluster(accempty_l);
           }
-          if (row >= a.M) continue;
+          if (nrows == 0) continue;  // warp-uniform
+          uint4 o1[4], o3[4], ou[4];
 #pragma unroll
           for (int c8 = 0; c8 < 32; c8 += 8) {
             uint32_t p1[4], p3[4], pu[4];
@@ -439,10 +484,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                 p3[j >> 1] = pack_f16x2(d3.x, d3.y);
                 pu[j >> 1] = pack_f16x2(u.x, u.y);
               }
-              const int64_t o = row * a.ldo + col + ph * 32 + c8;
-              *reinterpret_cast<uint4*>(static_cast<__half*>(a.out) + o) = make_uint4(p1[0], p1[1], p1[2], p1[3]);
-              *reinterpret_cast<uint4*>(static_cast<__half*>(a.out2) + o) = make_uint4(p3[0], p3[1], p3[2], p3[3]);
-              *reinterpret_cast<uint4*>(static_cast<__half*>(a.out3) + o) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+              o3[c8 >> 3] = make_uint4(p3[0], p3[1], p3[2], p3[3]);
+              ou[c8 >> 3] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
             } else {
 #pragma unroll
               for (int j = 0; j < 8; j += 2) {
@@ -450,11 +493,16 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
                 const float h3a = r * __uint_as_float(v3[c8 + j]), h3b = r * __uint_as_float(v3[c8 + j + 1]);
                 p1[j >> 1] = pack_bf16x2(silu_f(h1a) * h3a, silu_f(h1b) * h3b);
               }
-              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * a.ldo + col + ph * 32 + c8) =
-                  make_uint4(p1[0], p1[1], p1[2], p1[3]);
               (void)p3;
               (void)pu;
             }
+            o1[c8 >> 3] = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+          }
+          const int64_t ob = (row0 * a.ldo + col + ph * 32) * 2;  // byte offset of the warp's first row
+          warp_rows_out(tbuf, o1, static_cast<uint8_t*>(a.out) + ob, a.ldo * 2, nrows);
+          if constexpr (EPI == WG_SWIGLU_BWD) {
+            warp_rows_out(tbuf, o3, static_cast<uint8_t*>(a.out2) + ob, a.ldo * 2, nrows);
+            warp_rows_out(tbuf, ou, static_cast<uint8_t*>(a.out3) + ob, a.ldo * 2, nrows);
           }
         }
       } else if constexpr (EPI == WG_GATE) {

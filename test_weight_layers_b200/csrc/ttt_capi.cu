@@ -544,7 +544,7 @@ int launch_wgemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap
                  const CUtensorMap& b1, const WgArgs& args, int n_items, const Ws& w, cudaStream_t s) {
   if (n_items <= 0) return TTT_OK;
   auto k = k_wgemm<EPI, AMN, BMN>;
-  TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, WgLayout::ALLOC));
+  TTT_CHECK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, wg_smem_bytes<EPI>()));
   const int npairs = std::max(1, std::min(n_items, sm_count() / 2));
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -554,7 +554,7 @@ int launch_wgemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * npairs);
   cfg.blockDim = dim3(WG_THREADS);
-  cfg.dynamicSmemBytes = WgLayout::ALLOC;
+  cfg.dynamicSmemBytes = wg_smem_bytes<EPI>();
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
