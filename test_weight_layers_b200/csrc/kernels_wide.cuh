@@ -57,13 +57,11 @@ enum WgEpi : int {
   WG_NSOUT = 6         // Newton-Schulz product: C = alpha acc + beta Cin (fp32) and its bf16 hi/lo parts
 };
 
-// dynamic shared memory of an instance: the row-staging buffers only where the
-// epilogue stores 16-bit rows through them
+// dynamic shared memory of an instance: the row-staging buffers for every epilogue
+// but the fp32 split-K partials (written once per tile after the long K loop)
 template <int EPI>
 constexpr int wg_smem_bytes() {
-  return (EPI == WG_STORE16 || EPI == WG_STORE_BF16 || EPI == WG_SWIGLU_BWD || EPI == WG_SWIGLU_FWD)
-             ? WgLayout::ALLOC
-             : WgLayout::ALLOC_NO_TB;
+  return EPI != WG_PARTIAL ? WgLayout::ALLOC : WgLayout::ALLOC_NO_TB;
 }
 
 // Everything a launch needs besides the tensor maps.  Items are
@@ -509,6 +507,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
         // columns [tn*256 + half*128, +128) in four 32-column phases
         const int64_t col = (int64_t)it.tn * 256 + half * 128;
         const float ri = row < a.M ? a.rvec[row] : 0.f;
+        const int64_t row0 = row - lane;
+        const int nrows = (int)max((int64_t)0, min((int64_t)32, a.M - row0));
 #pragma unroll
         for (int ph = 0; ph < 4; ++ph) {
           uint32_t v[32];
@@ -518,7 +518,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
             tc_fence_before();
             warp_arrive_cluster(accempty_l);
           }
-          if (row >= a.M) continue;
+          if (nrows == 0) continue;  // warp-uniform
+          uint4 o[4];
 #pragma unroll
           for (int c8 = 0; c8 < 32; c8 += 8) {
             const uint4 q = pre[(ph * 32 + c8) >> 3];
@@ -530,15 +531,18 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
               const float ga = __uint_as_float(v[c8 + 2 * i]), gb = __uint_as_float(v[c8 + 2 * i + 1]);
               pk[i] = pack_bf16x2(xa * ri * silu_f(ga), xb * ri * silu_f(gb));
             }
-            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + row * a.ldo + col + ph * 32 + c8) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            o[c8 >> 3] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
+          warp_rows_out(tbuf, o, static_cast<uint8_t*>(a.out) + (row0 * a.ldo + col + ph * 32) * 2, a.ldo * 2, nrows);
         }
       } else if constexpr (EPI == WG_NSOUT) {
         // C = alpha acc + beta Cin for matrix h (rows M, stride ldo), plus C's bf16 hi and lo
         // parts (the next product's split operands), four 32-column phases
         const int64_t mbase = (int64_t)it.h * a.M * a.ldo + row * a.ldo + it.tn * 256 + half * 128;
         const float* cin = static_cast<const float*>(a.aux);
+        const int64_t row0 = row - lane;
+        const int nrows = (int)max((int64_t)0, min((int64_t)32, a.M - row0));
+        const int64_t wbase = mbase - (int64_t)lane * a.ldo;  // this warp's first row
 #pragma unroll
         for (int ph = 0; ph < 4; ++ph) {
           float4 ci[8];
@@ -553,6 +557,9 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
             tc_fence_before();
             warp_arrive_cluster(accempty_l);
           }
+          // fp32 C in two 16-column halves and its bf16 hi/lo parts, each through the
+          // staging buffer (rows of 64 bytes)
+          uint4 oc[2][4], oh[4], ol[4];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const float4 c = cin ? ci[q] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -561,8 +568,8 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
             o[1] = fmaf(a.alpha, __uint_as_float(v[4 * q + 1]), a.beta * c.y);
             o[2] = fmaf(a.alpha, __uint_as_float(v[4 * q + 2]), a.beta * c.z);
             o[3] = fmaf(a.alpha, __uint_as_float(v[4 * q + 3]), a.beta * c.w);
-            const int64_t off = mbase + ph * 32 + q * 4;
-            *reinterpret_cast<float4*>(static_cast<float*>(a.out) + off) = make_float4(o[0], o[1], o[2], o[3]);
+            oc[q >> 2][q & 3] = make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                                           __float_as_uint(o[3]));
             uint32_t hi[2], lo[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -570,9 +577,29 @@ __global__ void __launch_bounds__(WG_THREADS, 1)
               const float h0 = __uint_as_float(hi[e] << 16), h1 = __uint_as_float(hi[e] & 0xffff0000u);
               lo[e] = pack_bf16x2(o[2 * e] - h0, o[2 * e + 1] - h1);
             }
-            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out2) + off) = make_uint2(hi[0], hi[1]);
-            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out3) + off) = make_uint2(lo[0], lo[1]);
+            // 8 consecutive bf16 per uint4: q pairs (2k, 2k + 1) fill vector k
+            if (q & 1) {
+              oh[q >> 1].z = hi[0];
+              oh[q >> 1].w = hi[1];
+              ol[q >> 1].z = lo[0];
+              ol[q >> 1].w = lo[1];
+            } else {
+              oh[q >> 1].x = hi[0];
+              oh[q >> 1].y = hi[1];
+              ol[q >> 1].x = lo[0];
+              ol[q >> 1].y = lo[1];
+            }
           }
+          if (nrows == 0) continue;  // warp-uniform
+          const int64_t off = wbase + ph * 32;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+            warp_rows_out(tbuf, oc[hf], reinterpret_cast<uint8_t*>(static_cast<float*>(a.out) + off + hf * 16),
+                          a.ldo * 4, nrows);
+          warp_rows_out(tbuf, oh, reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(a.out2) + off), a.ldo * 2,
+                        nrows);
+          warp_rows_out(tbuf, ol, reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(a.out3) + off), a.ldo * 2,
+                        nrows);
         }
       }
     }
