@@ -213,10 +213,30 @@ __global__ void __launch_bounds__(256, RN <= 3 ? 3 : 2) k_prep_kv(const __nv_bfl
                                                     const float* __restrict__ eta,
                                                     const float* __restrict__ eta_part,
                                                     __half* __restrict__ Kh, __half* __restrict__ Vh, int64_t rows,
-                                                    int H, int d, int l2norm) {
+                                                    int H, int d, int l2norm, float* __restrict__ part_out) {
   constexpr int VN = 8;
+  // max|eta| from the block maxima of k_eta_absmax, or (part_out != nullptr, small
+  // calls) reduced here by every block over all rows * H values, block 0 then
+  // writing the maxima array the gradient kernel reads (its maximum first, zeros)
+  float emax;
+  if (part_out) {
+    __shared__ float red[8];
+    const int64_t n = rows * H;
+    float mx = 0.f;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) mx = fmaxf(mx, fabsf(__ldg(eta + i)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    emax = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) emax = fmaxf(emax, red[w]);
+    if (blockIdx.x == 0 && threadIdx.x < ETA_PARTS) part_out[threadIdx.x] = threadIdx.x == 0 ? emax : 0.f;
+  } else {
+    emax = eta_parts_max(eta_part);
+  }
   float vscale, inv_unused;  // V' = -s eta v with the value scale s of this call
-  value_scale(eta_parts_max(eta_part), vscale, inv_unused);
+  value_scale(emax, vscale, inv_unused);
   vscale = -vscale;
   const int lane = threadIdx.x & 31;
   const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;

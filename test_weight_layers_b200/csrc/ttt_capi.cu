@@ -468,18 +468,25 @@ int launch_eta_absmax(const float* eta, int64_t T, const ttt_dims& d, const Ws& 
 
 // fp16 gradient operands of T tokens (dense [T][H*d], written at kh, vh) from the
 // caller's bf16 K, V: K^ and V' = -s eta v with the value scale s of w.etapart.
+// self_max: the kernel reduces max|eta| itself and writes w.etapart (calls of at
+// most kSelfMaxEta values, where one launch fewer matters more than each block
+// reading all of eta); otherwise k_eta_absmax has written w.etapart.
+constexpr int64_t kSelfMaxEta = 8192;
 int launch_prep_kv(const void* K, int64_t ldk, const void* V, int64_t ldv, const float* eta, int64_t T,
-                   const ttt_dims& d, int l2norm, const Ws& w, __half* kh, __half* vh, cudaStream_t s) {
+                   const ttt_dims& d, int l2norm, const Ws& w, __half* kh, __half* vh, cudaStream_t s,
+                   bool self_max = false) {
   if (T == 0) return TTT_OK;
   ProfScope ps(TTT_PROF_NORM, s);
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((T * 32 + 255) / 256, (int64_t)sm_count() * 16));
   const int nvt = d.heads * d.d / 8;  // 16-byte vectors per row
+  const float* part_in = self_max ? nullptr : w.etapart;
+  float* part_out = self_max ? w.etapart : nullptr;
   if (nvt <= 96)
-    k_prep_kv<3><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, w.etapart,
-                                        kh, vh, T, d.heads, d.d, l2norm);
+    k_prep_kv<3><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, part_in,
+                                        kh, vh, T, d.heads, d.d, l2norm, part_out);
   else
-    k_prep_kv<4><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, w.etapart,
-                                        kh, vh, T, d.heads, d.d, l2norm);
+    k_prep_kv<4><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)K, ldk, (const __nv_bfloat16*)V, ldv, eta, part_in,
+                                        kh, vh, T, d.heads, d.d, l2norm, part_out);
   TTT_LAUNCHED();
   return TTT_OK;
 }
@@ -521,8 +528,9 @@ int prepare_update_operands(const void* K, int64_t ldk, const void* V, int64_t l
                             const ttt_dims& d, ttt_dtype dt, int l2norm, const Ws& w, cudaStream_t s,
                             UpdOperands* op) {
   if (dt == TTT_BF16) {
-    if (T > 0) TTT_TRY(launch_eta_absmax(eta, T, d, w, s));
-    TTT_TRY(launch_prep_kv(K, ldk, V, ldv, eta, T, d, l2norm, w, w.kh16, w.vh16, s));
+    const bool self_max = T * d.heads <= kSelfMaxEta;
+    if (T > 0 && !self_max) TTT_TRY(launch_eta_absmax(eta, T, d, w, s));
+    TTT_TRY(launch_prep_kv(K, ldk, V, ldv, eta, T, d, l2norm, w, w.kh16, w.vh16, s, self_max));
     const int64_t hd = (int64_t)d.heads * d.d;
     *op = {w.kh16, hd, w.vh16, hd, nullptr};
     return TTT_OK;
