@@ -203,7 +203,7 @@ def run_reference(args, cfg):
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    sample = 4096
+    sample = min(4096, cfg.tokens)
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
