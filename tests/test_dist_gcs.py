@@ -127,3 +127,55 @@ def test_two_rank_gcs_equals_single_process(chunk, steps, order, again):
     wr = np.concatenate([Wr.W1.ravel(), Wr.W3.ravel(), Wr.W2.ravel()])
     np.testing.assert_allclose(res[0][0], wr, rtol=0, atol=1e-10)
     np.testing.assert_allclose(np.vstack([res[0][1], res[1][1]]), Or, rtol=0, atol=1e-10)
+
+
+def _failing_rank_main(rank, world, port, out_q):
+    """Rank 1 fails inside its first gradient (an exception on the host, before the
+    collective); rank 0 must see its all-reduce fail rather than wait for ever."""
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=20))
+    W, K, V, Q, eta = _data()
+    H, d, m = W.dims
+    per = K.shape[0] // world
+    Kl, Vl, el = K[rank * per:(rank + 1) * per], V[rank * per:(rank + 1) * per], eta[rank * per:(rank + 1) * per]
+    state = {"W": W}
+
+    def grad(t0, t1):
+        if rank == 1:
+            raise RuntimeError("injected host-side failure")
+        g = O.grad(state["W"], O.l2norm_heads(Kl[t0:t1], H, d), Vl[t0:t1], el[t0:t1])
+        return torch.from_numpy(np.concatenate([g.W1.ravel(), g.W3.ravel(), g.W2.ravel()]))
+
+    def step(G):
+        pass
+
+    code = 0
+    try:
+        sharded_layer(per, 1, grad, lambda G: dist.all_reduce(G), step)
+        out_q.put((rank, "completed"))
+    except Exception as e:  # noqa: BLE001 - the test reports what each rank saw
+        out_q.put((rank, type(e).__name__))
+        code = 3 if rank == 1 else 0
+    out_q.close()
+    out_q.join_thread()  # the report is flushed before the process leaves
+    os._exit(code)  # no destroy_process_group: rank 1 leaves as a crashed rank would
+
+
+def test_a_failing_rank_surfaces_as_an_error_on_the_others():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    seen = {}
+    for _ in range(2):
+        r, what = q.get(timeout=120)
+        seen[r] = what
+    for p in procs:
+        p.join(timeout=60)
+    assert seen[1] == "RuntimeError"
+    # the surviving rank's collective raised (peer gone or timed out) instead of hanging
+    assert seen[0] != "completed", seen
+    assert procs[1].exitcode == 3
